@@ -1,0 +1,539 @@
+#!/usr/bin/env python
+"""Decode-attention benchmark of the ODA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl oda|reference]
+
+A step is one ODA decode step of the whole attention stack: Local attention with commit at
+every layer, the FP32 recall head and its gate, and the gated Full recompute with commit,
+as one CUDA-graph launch (liboda's step graph). The default workload is the long-context
+efficiency point: 28 layers (Qwen3-1.7B attention shapes: 16 query / 8 KV heads, head dim
+128), batch 1, 131072 prefilled tokens, s = 4, w = 2048, theta calibrated so that about
+12.5 % of steps recompute with Full. Inputs are seeded synthetic tensors (bf16 K/V/Q ~
+N(0, 1)) resident in HBM; the 15 GB KV cache is far larger than L2, so no flush is needed.
+
+Printed on rank 0: one JSON line with tokens/s (value), the KV bytes/s the step streams,
+the dominant kernel's roofline fraction, an end-to-end figure through the same API with
+host buffers, the clocks seen during the timed region and the fp64 oracle's CPU baseline.
+Under torchrun each rank runs its own sequences (no data-path collective: weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import oda_synth  # noqa: E402
+
+METRIC = "decode-attn tokens/s & achieved HBM GB/s (% of roofline) at 128K ctx, ρ≈12.5%"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "qwen3-1.7b-128k-b1"
+ROW_BYTES = 2 * 128 * 2          # K row + V row of one (position, KV head): 512 B
+PAGE_BYTES = 2 * 16 * 128 * 2    # K page + V page of one (page, KV head): 8 KB
+FALLBACK_HBM_GBS = 6650.0
+PROFILE = os.path.join(ROOT, "profiles", "decode_full_128k.md")
+KERNEL_SOURCES = ["oda_decode.cu", "oda_plan.cuh", "oda_common.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1024)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", choices=["oda", "reference"], default="oda")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(oda_synth.WORKLOADS))
+    ap.add_argument("--calib-steps", type=int, default=64)
+    ap.add_argument("--phase-steps", type=int, default=256)
+    ap.add_argument("--kernel-reps", type=int, default=28)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--quick", action="store_true",
+                    help="main timed region only (used for profiler launch lists)")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------------
+# Distributed plumbing: one process per GPU, each rank its own replica of the workload.
+# ---------------------------------------------------------------------------------------
+class Dist:
+    def __init__(self, gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64,
+                         device="cuda" if torch.cuda.is_available() else "cpu")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64,
+                         device="cuda" if torch.cuda.is_available() else "cpu")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------------
+# Clocks sampled during the timed region.
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", "oda_clocks_%d_%d.csv" % (os.getpid(), index))
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": seen, "samples": len(rows)}
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            return float(json.load(open(p))["hbm_gbs"]), "measured"
+        except (ValueError, KeyError):
+            pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "sparse_kv_recall_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(n_ctx_tokens_per_launch: float):
+    """DRAM bytes per Full launch from the committed ncu summary, scaled to this launch's
+    tokens; None when the summary is missing or was taken on other kernel sources."""
+    if not os.path.exists(PROFILE):
+        return None
+    info = {}
+    for line in open(PROFILE):
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            info[k.strip()] = v.strip().strip("`")
+    try:
+        if info.get("source_sha") != kernel_source_hash():
+            return None
+        per_token = float(info["dram_bytes_per_launch"]) / float(info["tokens_per_launch"])
+        return per_token * n_ctx_tokens_per_launch
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------------------
+# The product arm.
+# ---------------------------------------------------------------------------------------
+class Setup:
+    """Caches, recall head, engine and the resident pool of per-step inputs."""
+
+    def __init__(self, w, seed_offset: int, n_steps_total: int, theta: float, dev: str):
+        from sparse_kv_recall_b200.engine import OdaEngine, StagingLayout, fill_staging
+        self.w = oda_synth.scaled(w, seed=w.seed + 1000 * seed_offset)
+        w = self.w
+        self.lengths = oda_synth.prefill_lengths(w)
+        self.layout = oda_synth.make_layout(w, extra_tokens=n_steps_total + 4, device=dev)
+        self.caches = [oda_synth.make_kv_cache(w, self.layout, l, device=dev) for l in range(w.layers)]
+        rw = oda_synth.make_recall_weights(w, device=dev)
+        self.recall = (rw.w1, rw.b1, rw.w2, rw.b2)
+        self.eng = OdaEngine([c[0] for c in self.caches], [c[1] for c in self.caches],
+                             self.layout.block_table, w.num_q_heads, self.recall, theta,
+                             sink=w.sink, window=w.window)
+        self.eng.set_h_prev(oda_synth.make_h0(w, device=dev), 0)
+        lay = StagingLayout(w.layers, w.batch, w.num_q_heads, w.num_kv_heads, w.hidden)
+        self.slot = lay.nbytes
+        self.pool = torch.empty((n_steps_total, lay.nbytes), dtype=torch.uint8, device=dev)
+        for i in range(n_steps_total):
+            si = oda_synth.make_step_inputs(w, i, device=dev)
+            fill_staging(lay.views(self.pool[i]), si, [n + i + 1 for n in self.lengths])
+        torch.cuda.synchronize()
+
+    def feed(self, i: int):
+        self.eng.staging.copy_(self.pool[i], non_blocking=True)
+
+
+def launches_per_step(w, phases: int, steps: int) -> int:
+    """Kernels of this library launched by `steps` steps of which `phases` ran Full."""
+    return steps * (w.layers + 1) + phases * w.layers
+
+
+def run_oda(args, dist: Dist):
+    from sparse_kv_recall_b200 import build as B
+    from sparse_kv_recall_b200 import oda
+    B.build()
+    oda.load()
+    dev = "cuda:%d" % dist.local
+    torch.cuda.set_device(dist.local)
+    w = oda_synth.WORKLOADS[args.workload]
+    if w.mode != "oda":
+        raise SystemExit("bench.py times the ODA step; %s is a block-mask workload" % w.name)
+    K, W, C = args.steps, max(args.warmup, 3), args.calib_steps
+    if w.theta is not None:
+        C = 0
+    PH = 0 if args.quick else args.phase_steps
+    E2E = 0 if (args.quick or args.no_e2e) else min(K, 256)
+    total = C + W + K + PH + E2E
+    s = Setup(w, dist.rank, total, float("inf") if w.theta is None else w.theta, dev)
+    eng = s.eng
+    stream = torch.cuda.current_stream()
+    step = 0
+
+    # theta for the target Full-call rate: quantile of q over Local-only calibration steps
+    theta = w.theta
+    if theta is None:
+        qs = []
+        for _ in range(C):
+            s.feed(step)
+            eng.launch(step)
+            qs.append(eng.q_out.clone())
+            step += 1
+        q = torch.cat(qs).double().cpu().numpy()
+        theta = float(np.quantile(q, 1.0 - w.target_rho))
+        eng.set_theta(theta)
+
+    for _ in range(W):
+        s.feed(step)
+        eng.launch(step)
+        step += 1
+    torch.cuda.synchronize()
+
+    # ---- main timed region: K steps, inputs resident in HBM ----
+    fc0 = eng.full_count.clone()
+    st0 = eng.stats.clone()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        s.feed(step)
+        eng.launch(step)
+        step += 1
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    ms_local = e0.elapsed_time(e1)
+    ms = dist.max(ms_local)
+    fc = (eng.full_count - fc0).cpu().tolist()
+    st = (eng.stats - st0).cpu().tolist()
+    tokens_local = w.batch * K
+    tokens = dist.sum(tokens_local)
+    rho = fc[0] / float(w.batch * K)
+    kv_bytes = st[0] * ROW_BYTES
+    page_bytes = st[1] * PAGE_BYTES
+    launches = launches_per_step(w, fc[1], K)
+    peak, peak_kind = measured_peak()
+    result = {
+        "metric": METRIC, "value": tokens / (ms / 1e3), "unit": UNIT, "n_gpus": dist.world,
+        "steps": K, "warmup": W, "ms_per_step": ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "layers": w.layers, "batch_per_gpu": w.batch,
+                   "global_batch": w.batch * dist.world, "q_heads": w.num_q_heads,
+                   "kv_heads": w.num_kv_heads, "head_dim": 128, "prefill": w.prefill,
+                   "sink": w.sink, "window": w.window, "kv_dtype": "bf16",
+                   "rho_target": w.target_rho, "rho_realised": rho, "theta": theta,
+                   "calibration_steps": C, "l2": "no flush: 15 GB KV stream per Full step >> 126 MB L2"
+                   if w.name == DEFAULT_WORKLOAD else "no flush: KV working set > L2",
+                   "parallelism": "replicas (dp%d, no collective)" % dist.world},
+        "kv_stream": {"attended_bytes": kv_bytes, "gbs": kv_bytes / (ms_local / 1e3) / 1e9,
+                      "frac_of_peak": kv_bytes / (ms_local / 1e3) / 1e9 / peak,
+                      "page_bytes": page_bytes, "peak_gbs": peak, "peak_kind": peak_kind},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if args.quick:
+        return result, s
+
+    # ---- phase breakdown: same graphs with event nodes at the phase boundaries ----
+    eng.timing = True
+    eng.set_theta(theta)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(PH)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    fc0 = eng.full_count.clone()
+    gated = []
+    for i in range(PH):
+        before = eng.full_count[1].clone()
+        eng.set_events(step, evs[i])
+        s.feed(step)
+        eng.launch(step)
+        gated.append(before)
+        step += 1
+    torch.cuda.synchronize()
+    counts = torch.stack(gated).cpu().tolist() + [int(eng.full_count[1].item())]
+    ran_full = [counts[i + 1] > counts[i] for i in range(PH)]
+    t_local = [evs[i][0].elapsed_time(evs[i][1]) for i in range(PH)]
+    t_recall = [evs[i][1].elapsed_time(evs[i][2]) for i in range(PH)]
+    t_full = [evs[i][2].elapsed_time(evs[i][3]) for i in range(PH)]
+    t_step = [evs[i][0].elapsed_time(evs[i][3]) for i in range(PH)]
+    full_steps = [i for i in range(PH) if ran_full[i]]
+    local_steps = [i for i in range(PH) if not ran_full[i]]
+    mean = lambda xs: float(np.mean(xs)) if xs else None
+    T_step, T_loc = mean(t_step), mean(t_local)
+    T_full_exec = sum(t_full[i] for i in full_steps) / PH if PH else 0.0
+    gate_over = (T_step - T_loc - T_full_exec) / T_step if T_step else None
+    ctx = np.mean(s.lengths) + step - PH / 2
+    full_launch_bytes = w.batch * (ctx + 1) * w.num_kv_heads * ROW_BYTES
+    result["phases"] = {
+        "steps": PH, "steps_with_full": len(full_steps), "ms_step": T_step, "ms_local_phase": T_loc,
+        "ms_recall": mean(t_recall), "ms_full_phase_when_run": mean([t_full[i] for i in full_steps]),
+        "ms_full_phase_when_skipped": mean([t_full[i] for i in local_steps]),
+        "gate_overhead": gate_over,
+        "local_phase_kv_gbs": (w.batch * w.layers * w.num_kv_heads * (w.sink + w.window) * ROW_BYTES
+                               / (T_loc / 1e3) / 1e9) if T_loc else None,
+        "full_phase_kv_gbs": (w.layers * full_launch_bytes / (mean([t_full[i] for i in full_steps]) / 1e3)
+                              / 1e9) if full_steps else None,
+    }
+    eng.timing = False
+    eng.set_theta(theta)
+
+    # ---- dominant kernel alone: Full decode at this context, CUDA events per launch ----
+    from sparse_kv_recall_b200 import oda as O
+    ones = torch.ones(w.batch, dtype=torch.int32, device=dev)
+    out = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float32, device=dev)
+    q = eng.v["q_full_1" if w.layers > 1 else "q_full_0"]
+    kevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.kernel_reps)]
+    for r in range(3):
+        O.oda_decode_full(eng.kvs[r % w.layers], q, eng.scale, out, eng.decode_ws, gate=ones)
+    torch.cuda.synchronize()
+    for r, (a, b) in enumerate(kevs):
+        a.record(stream)
+        O.oda_decode_full(eng.kvs[r % w.layers], q, eng.scale, out, eng.decode_ws, gate=ones)
+        b.record(stream)
+    torch.cuda.synchronize()
+    dur = float(np.mean([a.elapsed_time(b) for a, b in kevs]))
+    ctx_tokens = int(eng.seq_lens.sum().item())
+    alg = ctx_tokens * w.num_kv_heads * ROW_BYTES
+    achieved = alg / (dur / 1e3) / 1e9
+    traffic = profiled_traffic(ctx_tokens)
+    result["roofline"] = {"kernel": "oda_decode_full (decode_kernel<%d>)" % w.group,
+                          "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                          "frac": achieved / peak, "traffic": traffic,
+                          "algorithmic_bytes": alg, "ms_per_launch": dur,
+                          "peak_kind": peak_kind + " (burst copy; kernel timed alone)"}
+
+    # ---- end to end through the same API: host inputs in, selected output out ----
+    if E2E:
+        host_pool = torch.empty((E2E, s.slot), dtype=torch.uint8, pin_memory=True)
+        host_pool.copy_(s.pool[step:step + E2E])
+        out_h = torch.empty((2, w.batch, w.hidden), dtype=torch.float32, pin_memory=True)
+        gate_h = torch.empty((2, w.batch), dtype=torch.int32, pin_memory=True)
+        torch.cuda.synchronize()
+        dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(E2E):
+            eng.staging.copy_(host_pool[i], non_blocking=True)
+            eng.launch(step)
+            out_h[i % 2].copy_(eng.selected_last(step), non_blocking=True)
+            gate_h[i % 2].copy_(eng.gate, non_blocking=True)
+            step += 1
+        b.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        ms_e2e = dist.max(a.elapsed_time(b))
+        result["e2e"] = {"value": dist.sum(w.batch * E2E) / (ms_e2e / 1e3), "unit": UNIT,
+                         "h2d_bytes_per_step": s.slot,
+                         "d2h_bytes_per_step": w.batch * (w.hidden * 4 + 4)}
+    assert int(eng.status.item()) == 0, "device status %d" % int(eng.status.item())
+    return result, s
+
+
+# ---------------------------------------------------------------------------------------
+# The fp64 oracle on the host: the CPU baseline leg and the reference arm.
+# ---------------------------------------------------------------------------------------
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+class OracleSampler:
+    """Times the oracle on bounded pieces of one decode step of the workload and
+    extrapolates to a whole step: Local at one layer (all heads), the recall head, and Full
+    at one layer for one KV head (its G query heads) over one of `chunks` equal slices of the
+    history (sample i takes slice i mod chunks; the oracle's cost is linear in positions);
+    a step costs L * local + recall + rho * L * Hkv * chunks * full_slice."""
+
+    def __init__(self, w, rho: float, dev: str, chunks: int = 1):
+        self.chunks = chunks
+        from oracle import oda_oracle as O
+        self.O, self.w, self.rho = O, w, rho
+        lay = oda_synth.make_layout(w, extra_tokens=8, device=dev)
+        kc, vc = oda_synth.make_kv_cache(w, lay, 0, device=dev)
+        self.kbits, self.vbits = oda_synth.bf16_bits(kc), oda_synth.bf16_bits(vc)
+        del kc, vc
+        self.bt = lay.block_table.cpu().numpy()
+        self.t = oda_synth.prefill_lengths(w)[0]
+        g = torch.Generator().manual_seed(w.seed)
+        self.q = torch.randn((w.num_q_heads, 128), generator=g).to(torch.bfloat16)
+        self.qbits = oda_synth.bf16_bits(self.q)
+        rw = oda_synth.make_recall_weights(w)
+        self.rec = [x.double().numpy() for x in (rw.w1, rw.b1, rw.w2)] + [rw.b2]
+        self.h = np.random.default_rng(0).standard_normal((3, w.batch, w.hidden))
+
+    def sample(self, i: int) -> float:
+        """Seconds of one extrapolated oracle decode step (per sequence of the batch)."""
+        O, w = self.O, self.w
+        G = w.num_q_heads // w.num_kv_heads
+        qf = O.widen_bf16(self.qbits)
+        t0 = time.perf_counter()
+        pos = O.local_positions(self.t, w.sink, w.window)
+        ks = [O.paged_rows(self.kbits, self.bt[0], pos, g) for g in range(w.num_kv_heads)]
+        vs = [O.paged_rows(self.vbits, self.bt[0], pos, g) for g in range(w.num_kv_heads)]
+        O.decode_attention(qf, ks, vs, 1 / math.sqrt(128))
+        t1 = time.perf_counter()
+        O.recall_score(self.h[0], self.h[1], self.h[2], *self.rec)
+        t2 = time.perf_counter()
+        g = i % w.num_kv_heads
+        pos = np.array_split(O.full_positions(self.t), self.chunks)[i % self.chunks]
+        kr = O.paged_rows(self.kbits, self.bt[0], pos, g)
+        vr = O.paged_rows(self.vbits, self.bt[0], pos, g)
+        O.decode_attention(qf[g * G:(g + 1) * G], [kr], [vr], 1 / math.sqrt(128))
+        t3 = time.perf_counter()
+        per_seq = (w.layers * (t1 - t0)
+                   + self.rho * w.layers * w.num_kv_heads * self.chunks * (t3 - t2))
+        return w.batch * per_seq + (t2 - t1)
+
+
+def cpu_baseline(w, rho: float, dev: str, budget_s: float = 20.0) -> dict:
+    s = OracleSampler(w, rho, dev)
+    spent, n, total = 0.0, 0, 0.0
+    while spent < budget_s and n < 64:
+        a = time.perf_counter()
+        total += s.sample(n)
+        spent += time.perf_counter() - a
+        n += 1
+    return {"value": w.batch * n / total, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": ("%d oracle samples of one %s decode step (Local at one layer, recall, Full "
+                       "at one layer for one KV head), extrapolated to all %d layers, %d KV heads "
+                       "and rho=%.3f; %.1f s of CPU time" % (n, w.name, w.layers, w.num_kv_heads,
+                                                             rho, spent))}
+
+
+def run_reference(args, dist: Dist):
+    """The oracle, as it stands, timed on the host cores on this workload."""
+    if dist.rank != 0:
+        return None
+    w = oda_synth.WORKLOADS[args.workload]
+    rho = w.target_rho if w.target_rho is not None else 0.5
+    dev = "cuda:%d" % dist.local if torch.cuda.is_available() else "cpu"
+    s = OracleSampler(w, rho, dev, chunks=16)
+    for i in range(max(args.warmup, 3)):
+        s.sample(i)
+    wall = time.perf_counter()
+    total = sum(s.sample(i) for i in range(args.steps))
+    wall = time.perf_counter() - wall
+    value = w.batch * args.steps / total
+    cores = _blas_threads()
+    sample = ("each step: one oracle sample of a %s decode step (Local at one layer, recall, "
+              "Full at one layer for one KV head over 1/16 of the history) extrapolated to %d "
+              "layers, %d KV heads, the whole history and rho=%.3f"
+              % (w.name, w.layers, w.num_kv_heads, rho))
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "rho": rho},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample + "; %.1f s wall" % wall},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    dist = Dist(args.gpus)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, dist)
+        else:
+            res, setup = run_oda(args, dist)
+            if dist.rank == 0 and dist.world == 1 and not (args.no_cpu_baseline or args.quick):
+                rho = res["config"]["rho_realised"]
+                del setup
+                torch.cuda.empty_cache()
+                res["cpu_baseline"] = cpu_baseline(oda_synth.WORKLOADS[args.workload], rho,
+                                                   "cuda:%d" % dist.local)
+        if res is not None and dist.rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,222 @@
+/*
+ * oda.h -- C ABI of liboda, the sm_100a (B200) decode hot path of On-Demand Attention (ODA)
+ * and of Declarative Attention's block-granular keep masks.
+ *
+ * Sources:
+ *   [ODA] "On-Demand Attention: Language Models Know When to Recall" (arxiv-wiki summary):
+ *         sections 접근 방법 (approach), 주요 결과 (results), 개발자 관점 (developer view).
+ *   [DA]  "[논문리뷰] Language Models Can Control Their Own Attention", section 3 (method).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensors are caller-owned device memory (the library allocates nothing on the decode
+ *     path and keeps no pointer after a call returns). Layouts are dense row-major.
+ *   - Every compute call is asynchronous on `stream` (a cudaStream_t / CUstream handle; NULL
+ *     = legacy default stream) and never synchronises the host, so it can be captured in a
+ *     CUDA graph.
+ *   - Host-side checks return ODA_OK (0) or a negative ODA_ERR_* code before anything is
+ *     launched; nothing is thrown across the ABI.
+ *   - Errors that only the device can see (a bad page id, a bad length, a bad keep list, a
+ *     wait that ran out) are written to oda_kv.dev_status (first error wins) and the
+ *     offending work item is skipped; kernels never trap.
+ *   - Head dimension 128, page size 16 tokens, bf16 K/V/Q, fp32 accumulation. Query head h
+ *     reads KV head h / (num_q_heads / num_kv_heads); the group size must be 1, 2 or 4.
+ */
+#ifndef ODA_H_
+#define ODA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------------------------- */
+enum {
+  ODA_OK = 0,
+  ODA_ERR_INVALID_ARG = -1,       /* null pointer, negative size, unknown enum value        */
+  ODA_ERR_UNSUPPORTED_SHAPE = -2, /* head_dim != 128, block_size != 16, bad GQA group, ... */
+  ODA_ERR_WORKSPACE_TOO_SMALL = -3,
+  ODA_ERR_CUDA = -4,              /* a CUDA runtime call (launch, graph build) failed       */
+  ODA_ERR_NOT_IMPLEMENTED = -5,
+  /* device-side codes, written to oda_kv.dev_status */
+  ODA_DEV_BAD_BLOCK = 1,          /* a page id outside [0, num_blocks): page skipped        */
+  ODA_DEV_BAD_LEN = 2,            /* seq_lens[b] < 1 or beyond the page table: sequence
+                                     treated as empty                                      */
+  ODA_DEV_BAD_KEEP_LIST = 3,      /* keep entry not strictly ascending or after page t/16,
+                                     or keep_counts[b] outside [0, max_keep]: entry skipped */
+  ODA_DEV_TIMEOUT = 4             /* a bounded device wait gave up                          */
+};
+
+enum { ODA_F32 = 0, ODA_BF16 = 1 };                               /* output / input dtypes */
+enum { ODA_MODE_LOCAL = 0, ODA_MODE_FULL = 1, ODA_MODE_KEEP = 2 }; /* visible-set rules    */
+enum { ODA_STAT_ROWS = 0, ODA_STAT_PAGES = 1, ODA_STATS_LEN = 2 };
+
+/* Returns a static, human-readable name for any status code above. */
+const char* oda_status_string(int code);
+
+/* Library ABI version (major * 100 + minor). */
+int oda_version(void);
+
+/* ---- the paged KV cache ([ODA] 개발자 관점: the runtime keeps the whole history paged, with a
+ *      Local view and a Full view over the same cache) ---------------------------------- */
+typedef struct {
+  void* k_cache;                /* bf16 [num_blocks][num_kv_heads][block_size][head_dim]    */
+  void* v_cache;                /* same layout; each (page, KV head) is one 4 KB run         */
+  const int32_t* block_table;   /* int32 [batch][max_blocks_per_seq]: physical page of each
+                                   logical page; only entries < ceil(seq_len/16) are read   */
+  const int32_t* seq_lens;      /* int32 [batch]: tokens in the cache INCLUDING the current
+                                   one, i.e. t + 1 for current position t                   */
+  int32_t batch;
+  int32_t num_kv_heads;
+  int32_t head_dim;             /* must be 128                                              */
+  int32_t block_size;           /* must be 16                                               */
+  int32_t max_blocks_per_seq;
+  int32_t num_blocks;
+  int32_t* dev_status;          /* nullable device int32: first ODA_DEV_* error (0 = none)  */
+  unsigned long long* stats;    /* nullable device u64[ODA_STATS_LEN]: [ROWS] += visible
+                                   (position, KV head) rows attended, [PAGES] += (page, KV
+                                   head) pairs streamed from HBM                            */
+} oda_kv;
+
+/* Bytes of workspace the decode calls need for `batch` sequences on the current device. The
+ * workspace holds split partials and merge tickets; it must be zero-filled once before its
+ * first use and is left zero-filled by every call, so one buffer serves any number of calls
+ * issued in stream order. Returns ODA_OK or an error code. */
+int oda_decode_workspace_size(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads,
+                              size_t* bytes);
+
+/* ---- K1: commit of the step's K/V ([ODA] 접근 방법: the selected path's current-position
+ *      K/V joins the fully retained history) -------------------------------------------
+ * Writes k_new[b][h][:] and v_new[b][h][:] (bf16 [batch][num_kv_heads][head_dim]) into slot
+ * t = seq_lens[b] - 1 of every KV head, through block_table[b][t / 16], row t % 16. With a
+ * non-null gate (int32 [batch]) only sequences with gate[b] != 0 are written, overwriting
+ * what the Local pass committed: this is the commit of the Full result. */
+int oda_kv_append(const oda_kv* kv, const void* k_new, const void* v_new,
+                  const int32_t* gate, void* stream);
+
+/* ---- K2 + K3: decode attention, split over the whole GPU and merged in-kernel ----------
+ * For every sequence b and query head h: out[b][h] = softmax(scale * K q) V over the visible
+ * positions of KV head h / G, with the natural-log normaliser in lse[b][h] (nullable).
+ *   q   : bf16 [batch][num_q_heads][128]
+ *   out : [batch][num_q_heads][128], fp32 (out_dtype = ODA_F32) or bf16 (ODA_BF16)
+ *   lse : fp32 [batch][num_q_heads] or NULL
+ *   ws  : workspace of at least oda_decode_workspace_size() bytes (zeroed once)
+ * An empty visible set gives out = 0 and lse = -inf. */
+
+/* Local ([ODA] 접근 방법, decoding procedure; 주요 결과, last item): the first `sink`
+ * positions plus the `window` most recent ones, the current position included, as a set
+ * union. With non-null k_new / v_new (bf16 [batch][num_kv_heads][128]) the call also
+ * commits them at slot t (as oda_kv_append would) and attends to them there. */
+int oda_decode_local(const oda_kv* kv, const void* q, int32_t num_q_heads, int32_t sink,
+                     int32_t window, float scale, const void* k_new, const void* v_new,
+                     void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Full ([ODA] 접근 방법: recompute the step over the whole history from the same prior
+ * state): positions 0..t. With a non-null gate (int32 [batch]) sequences with gate[b] == 0
+ * are skipped entirely -- no KV byte is read and out/lse rows keep their contents -- and the
+ * GPU's work is balanced over the gated sequences only. Non-null k_new / v_new commit the
+ * Full K/V at slot t for the gated sequences (overwriting the Local commit). */
+int oda_decode_full(const oda_kv* kv, const void* q, int32_t num_q_heads, float scale,
+                    const int32_t* gate, const void* k_new, const void* v_new,
+                    void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/* Keep-block mask ([DA] section 3: the engine rewrites the block table so that only the kept
+ * pages reach the attention kernel). keep_blocks: int32 [batch][max_keep] logical page ids,
+ * strictly ascending, each <= t / 16; keep_counts: int32 [batch]. Visible positions are the
+ * kept pages' positions up to t. The rewrite (logical -> physical page) happens inside the
+ * kernel's address generation; no compacted table is materialised. */
+int oda_decode_blockmask(const oda_kv* kv, const void* q, int32_t num_q_heads, float scale,
+                         const int32_t* keep_blocks, const int32_t* keep_counts,
+                         int32_t max_keep, void* out, int32_t out_dtype, float* lse,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Debug export of the visibility plan the decode kernels use: mask[b][p] = 1 where position
+ * p < max_tokens is visible to sequence b under `mode` (ODA_MODE_*), 0 elsewhere (uint8
+ * [batch][max_tokens], fully written). gate (nullable) applies to ODA_MODE_FULL as in
+ * oda_decode_full; keep_* apply to ODA_MODE_KEEP. */
+int oda_visible_mask(const oda_kv* kv, int32_t mode, int32_t sink, int32_t window,
+                     const int32_t* gate, const int32_t* keep_blocks,
+                     const int32_t* keep_counts, int32_t max_keep, uint8_t* mask,
+                     int32_t max_tokens, void* stream);
+
+/* ---- K4: recall head and gate ([ODA] 접근 방법: q_t = R(h_{t-1}, E(x_t), h^L_t); Full iff
+ *      q_t > theta; 개발자 관점: evaluated in FP32 on the GPU, no routing sync) ----------
+ *   h_prev  : fp32 [batch][hidden]  previous step's selected last-layer output
+ *   emb     : fp32 [batch][hidden]  embedding of the current token
+ *   h_local : [batch][hidden], fp32 or bf16 (h_local_dtype): this step's last-layer Local out
+ *   w1      : fp32 [3 * hidden][mlp] (rows: h_prev, then emb, then h_local); b1, w2: fp32 [mlp]
+ * z = w1^T [h_prev; emb; h_local] + b1, q = w2 . GELU(z) + b2 (exact erf GELU).
+ * Writes q_out (fp32 [batch]) and gate_out (int32 [batch], 1 iff q > theta); if full_count
+ * (nullable u64[2]) is given, adds the number of gated sequences to full_count[0] and 1 to
+ * full_count[1] when at least one sequence is gated; and, if graph_cond_handle != 0 (a
+ * cudaGraphConditionalHandle), sets that graph condition to 1 iff any sequence is gated.
+ * mlp must be a multiple of 64; hidden >= 1. ws: oda_recall_workspace_size() bytes, zeroed
+ * once and left zeroed. */
+int oda_recall_workspace_size(int32_t batch, int32_t hidden, int32_t mlp, size_t* bytes);
+int oda_recall_score(const float* h_prev, const float* emb, const void* h_local,
+                     int32_t h_local_dtype, int32_t batch, int32_t hidden, int32_t mlp,
+                     const float* w1, const float* b1, const float* w2, float b2, float theta,
+                     float* q_out, int32_t* gate_out, unsigned long long* full_count,
+                     unsigned long long graph_cond_handle, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* ---- Step runtime: one whole ODA decode step as one CUDA graph ([ODA] 개발자 관점: Local,
+ *      the FP32 recall head and the conditional Full recompute in one GPU execution stream,
+ *      e.g. CUDA Graphs) ----------------------------------------------------------------
+ * The graph runs, per launch: Local (with commit) at every layer; the recall head on the last
+ * layer's Local output; then, inside a conditional IF node that the recall head opens only
+ * when some sequence is gated, Full (with gated commit) at every layer not marked local-only.
+ * All pointers are captured at creation: the caller refreshes the buffers' contents (seq_lens
+ * advanced by one, new q/k/v, new embedding) between launches. */
+typedef struct oda_step_graph oda_step_graph;
+
+typedef struct {
+  int32_t num_layers;
+  const oda_kv* layers;               /* host array [num_layers]; per-layer k/v caches, the
+                                          same block_table, seq_lens and shapes             */
+  int32_t num_q_heads;
+  int32_t sink, window;
+  float scale;
+  const void* const* q_local;          /* host arrays [num_layers] of device pointers, bf16  */
+  const void* const* k_local;
+  const void* const* v_local;
+  const void* const* q_full;
+  const void* const* k_full;
+  const void* const* v_full;
+  void* const* out;                    /* [num_layers] fp32 [batch][Hq][128]: selected out   */
+  float* const* lse;                   /* nullable; else [num_layers] fp32 [batch][Hq]       */
+  const int32_t* local_only;           /* nullable host int32 [num_layers]: 1 = the layer never
+                                          recomputes with Full (hybrid backbones)           */
+  const float* h_prev;                 /* fp32 [batch][Hq*128], read by the recall head      */
+  const float* emb;                    /* fp32 [batch][Hq*128]                               */
+  const float* w1;                     /* recall head, as in oda_recall_score                */
+  const float* b1;
+  const float* w2;
+  float b2;
+  float theta;
+  int32_t mlp;
+  float* q_out;                        /* fp32 [batch]                                      */
+  int32_t* gate_out;                   /* int32 [batch]                                     */
+  unsigned long long* full_count;      /* nullable u64[2], as in oda_recall_score            */
+  void* decode_ws;  size_t decode_ws_bytes;
+  void* recall_ws;  size_t recall_ws_bytes;
+  int32_t use_conditional;             /* 1: IF node around the Full phase; 0: Full kernels
+                                          always launch and skip ungated sequences on-device */
+  int32_t timing_events;               /* 1: event-record nodes at phase boundaries          */
+} oda_step_desc;
+
+int oda_step_graph_create(const oda_step_desc* desc, void* stream, oda_step_graph** graph);
+int oda_step_graph_launch(oda_step_graph* graph, void* stream);
+/* With timing_events = 1: point the graph's four phase events (step start, Local done, recall
+ * done, Full done) at caller-created cudaEvent_t handles for the next launches. */
+int oda_step_graph_set_events(oda_step_graph* graph, void* ev_start, void* ev_local,
+                              void* ev_recall, void* ev_end);
+void oda_step_graph_destroy(oda_step_graph* graph);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ODA_H_ */

@@ -123,13 +123,15 @@ class PagedLayout:
     capacity: list               # tokens each sequence can hold
 
 
-def make_layout(w: Workload, extra_tokens: int, device="cpu") -> PagedLayout:
-    """Hand out physical pages for n_b + extra_tokens tokens per sequence, in a seeded
-    random order over the whole pool."""
-    lens = prefill_lengths(w)
+def make_layout(w: Workload, extra_tokens: int, device="cpu", lengths=None,
+                spare_pages: int = 0) -> PagedLayout:
+    """Hand out physical pages for n_b + extra_tokens tokens per sequence (n_b from the
+    workload, or the explicit `lengths`), in a seeded random order over the whole pool;
+    `spare_pages` extra pages stay unassigned."""
+    lens = list(lengths) if lengths is not None else prefill_lengths(w)
     caps = [n + extra_tokens for n in lens]
     per_seq = [math.ceil(c / w.block_size) for c in caps]
-    total = sum(per_seq)
+    total = sum(per_seq) + spare_pages
     maxb = max(per_seq)
     perm = torch.randperm(total, generator=_gen(w.seed, _P_BLOCKTABLE)).to(torch.int32)
     bt = torch.full((w.batch, maxb), -1, dtype=torch.int32)

@@ -1,0 +1,738 @@
+// K2 + K3: paged decode attention for Local, Full and keep-page visibility, split over the
+// whole GPU and merged inside the same launch.
+//
+// Work decomposition. Every sequence b contributes npages(b) visible pages per KV head; the
+// flattened list of (b, KV head g, page j) units is cut into gridDim.x equal contiguous
+// shares, one per CTA (grid = 2 CTAs per SM, one wave, no tail). A share may cover part of
+// one (b, g) or the ends of several. Inside a CTA each of the 4 warps streams every 4th page
+// of the current (b, g) piece through its own 3-stage ring of shared-memory stages filled by
+// 1-D bulk copies (TMA engine, 4 KB K page + 4 KB V page per stage), and keeps an online
+// softmax for all G = Hq / Hkv query heads that share the KV head, so each page is read
+// from HBM once for the whole group. A piece's 8 half-warp states are merged in shared
+// memory; if the (b, g) spans several CTAs, each writes its normalised partial (O, log2-sum)
+// to the workspace and the last to arrive (atomic ticket) merges them in fixed order.
+//
+// Lane layout for a 16 x 128 page: lane = 16 * half + li; lane li owns dims [8 li, 8 li + 8)
+// of rows 2k + half, k = 0..7. Dot products are reduced over the 16 lanes of a half by a
+// reduce-scatter butterfly, after which lane li holds row 2 (li / 2) + half for heads
+// (li % 2) * G / 2 + u.
+#include <math.h>
+
+#include "oda_plan.cuh"
+
+namespace oda {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;   // == kHeadDim: merges map one thread to one dim
+constexpr int kStages = 3;
+constexpr int kStageBytes = 2 * kPageBytes;
+constexpr int kCtasPerSm = 2;
+constexpr int kMaxBatch = 1024;
+constexpr int kMaxGroup = 4;
+
+static_assert(kThreads == kHeadDim, "merge maps one thread per output dim");
+
+struct DecodeParams {
+  PlanArgs plan;
+  const __nv_bfloat16* k_cache;
+  const __nv_bfloat16* v_cache;
+  __nv_bfloat16* k_cache_w;
+  __nv_bfloat16* v_cache_w;
+  int batch, hkv, hq;
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k_new;  // nullable: commit at slot t
+  const __nv_bfloat16* v_new;
+  float scale_log2;            // scale * log2(e): scores are kept in base-2 units
+  void* out;
+  int out_bf16;
+  float* lse;
+  float* ws_o;                 // [slots][G][128]
+  float* ws_lse;               // [slots][G], base-2 log-sum
+  unsigned int* ws_ticket;     // [batch * hkv]
+  int* status;
+  unsigned long long* stats;
+};
+
+// ---- reduce-scatter of C values over the 16 lanes of a half-warp ------------------------
+// After the call, v[0 .. max(C/16, 1)) of lane li hold the sums of the original value
+// indices li * (C / 16) + u (for C < 16 the last steps are plain all-reduces).
+template <int C, int O>
+__device__ __forceinline__ void reduce_scatter(float* v, int lane) {
+  if constexpr (O >= 1) {
+    if constexpr (C > 1) {
+      const bool up = (lane & O) != 0;
+#pragma unroll
+      for (int j = 0; j < C / 2; ++j) {
+        const float send = up ? v[j] : v[j + C / 2];
+        const float keep = up ? v[j + C / 2] : v[j];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+      }
+      reduce_scatter<C / 2, O / 2>(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+      reduce_scatter<1, O / 2>(v, lane);
+    }
+  }
+}
+
+template <int G>
+struct Vpl {
+  static constexpr int value = G >= 2 ? G / 2 : 1;  // softmax values each lane owns
+};
+
+// One page: scores, online-softmax update, P.V accumulation.
+template <int G>
+__device__ __forceinline__ void page_step(const unsigned char* stage, const float (&qf)[G][8],
+                                          float (&m_run)[Vpl<G>::value],
+                                          float (&l_run)[Vpl<G>::value], float (&acc)[G][8],
+                                          float* ps, const SeqPlan& sp, int lp, int lane,
+                                          unsigned& rows_vis) {
+  constexpr int VPL = Vpl<G>::value;
+  const int half = lane >> 4, li = lane & 15;
+  const uint4* K = reinterpret_cast<const uint4*>(stage);
+  const uint4* V = reinterpret_cast<const uint4*>(stage + kPageBytes);
+
+  float sc[8 * G];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float kf[8];
+    unpack8(K[(2 * k + half) * 16 + li], kf);
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s = fmaf(qf[gg][e], kf[e], s);
+      sc[k * G + gg] = s;
+    }
+  }
+  reduce_scatter<8 * G, 8>(sc, lane);
+
+  const int myk = li >> 1;
+  const bool vis = row_visible(sp, lp * kPage + 2 * myk + half);
+  rows_vis += __popc(__ballot_sync(0xffffffffu, vis) & 0x55555555u);
+
+  float* pshare = ps;                 // [2 halves][8 rows][G]
+  float* ashare = ps + 16 * G;        // [2 halves][G]
+#pragma unroll
+  for (int u = 0; u < VPL; ++u) {
+    const float v = vis ? sc[u] : -INFINITY;
+    float mx = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mnew = fmaxf(m_run[u], mx);
+    const float pr = (v == -INFINITY) ? 0.f : exp2f(v - mnew);
+    const float al = (m_run[u] == mnew) ? 1.f : exp2f(m_run[u] - mnew);
+    l_run[u] = l_run[u] * al + pr;
+    m_run[u] = mnew;
+    const int gh = (G >= 2) ? ((li & 1) * (G / 2) + u) : 0;
+    if (G >= 2 || (li & 1) == 0) {
+      pshare[(half * 8 + myk) * G + gh] = pr;
+      if (myk == 0) ashare[half * G + gh] = al;
+    }
+  }
+  __syncwarp();
+
+#pragma unroll
+  for (int gg = 0; gg < G; ++gg) {
+    const float al = ashare[half * G + gg];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[gg][e] *= al;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float vf[8];
+    unpack8(V[(2 * k + half) * 16 + li], vf);
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      const float pk = pshare[(half * 8 + k) * G + gg];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[gg][e] = fmaf(pk, vf[e], acc[gg][e]);
+    }
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void store_out(const DecodeParams& p, size_t idx, float v) {
+  if (p.out_bf16)
+    reinterpret_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<float*>(p.out)[idx] = v;
+}
+
+// Final output of query heads g*G .. g*G+G-1 of sequence b; thread tid writes dim tid.
+template <int G>
+__device__ __forceinline__ void write_final(const DecodeParams& p, int b, int g,
+                                            const float (&o)[G], const float (&lse2)[G]) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int gg = 0; gg < G; ++gg) {
+    const size_t h = (size_t)b * p.hq + g * G + gg;
+    store_out(p, h * kHeadDim + tid, o[gg]);
+    if (p.lse != nullptr && tid == 0)
+      p.lse[h] = (lse2[gg] == -INFINITY) ? -INFINITY : lse2[gg] * 0.69314718055994531f;
+  }
+}
+
+// CTA whose share contains flattened unit x (shares are [c*T/P, (c+1)*T/P), P <= T).
+__device__ __forceinline__ int cta_of(long long x, long long T, int P) {
+  return (int)(((x + 1) * P - 1) / T);
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecodeParams p) {
+  constexpr int VPL = Vpl<G>::value;
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned char* stages = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * kStageBytes);
+  float* pscratch = reinterpret_cast<float*>(bars + kWarps * kStages);
+  constexpr int kPs = 18 * G;  // per-warp softmax exchange: 16 G weights + 2 G rescales
+  int* pre = reinterpret_cast<int*>(pscratch + kWarps * kPs);  // [batch + 1] prefix of units
+  __shared__ int s_last;
+  __shared__ unsigned long long s_rows, s_pages;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int half = lane >> 4, li = lane & 15;
+  const int B = p.batch, Hkv = p.hkv;
+  const int P = gridDim.x, c = blockIdx.x;
+
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[warp * kStages + s], 1);
+    fence_barrier_init();
+  }
+  if (tid == 0) {
+    s_rows = 0;
+    s_pages = 0;
+    pre[0] = 0;
+  }
+  for (int b = tid; b < B; b += kThreads) {
+    const SeqPlan sp = make_plan(p.plan, b);
+    pre[b + 1] = sp.npages * Hkv;
+    if (c == 0) {
+      if (sp.bad_len) report(p.status, ODA_DEV_BAD_LEN);
+      if (sp.bad_keep) report(p.status, ODA_DEV_BAD_KEEP_LIST);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {  // inclusive scan of the per-sequence unit counts
+    int carry = 0;
+    for (int base = 0; base < B; base += 32) {
+      const int i = base + lane;
+      int v = i < B ? pre[i + 1] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+      }
+      v += carry;
+      if (i < B) pre[i + 1] = v;
+      carry = __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
+  __syncthreads();
+  const long long T = pre[B];
+
+  // Sequences with nothing visible (bad length, empty keep list) but not gated off.
+  for (int bg = c; bg < B * Hkv; bg += P) {
+    const int b = bg / Hkv;
+    if (pre[b + 1] == pre[b] && !(p.plan.gate != nullptr && p.plan.gate[b] == 0)) {
+      float o[G], l2[G];
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        o[gg] = 0.f;
+        l2[gg] = -INFINITY;
+      }
+      write_final<G>(p, b, bg % Hkv, o, l2);
+    }
+  }
+
+  const uint64_t policy = l2_evict_first_policy();
+  unsigned char* wst = stages + warp * kStages * kStageBytes;
+  uint64_t* wbar = bars + warp * kStages;
+  float* ps = pscratch + warp * kPs;
+  unsigned wcount = 0;       // pages this warp has consumed, over all pieces
+  bool dead = false;         // a bounded wait gave up: stop touching the ring
+  unsigned rows_vis = 0, pages_read = 0;
+
+  // Shares go to the first Pe = min(P, T) CTAs only, so that every CTA holding a share has
+  // at least one unit and the CTAs that touch a (b, g) are exactly a contiguous index range.
+  const int Pe = (int)min((long long)P, T);
+  long long x = c < Pe ? (T * c) / Pe : 0;
+  const long long x_end = c < Pe ? (T * (c + 1)) / Pe : 0;
+  while (x < x_end) {
+    int lo = 0, hi = B - 1;  // largest b with pre[b] <= x
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    const int npg = (pre[b + 1] - pre[b]) / Hkv;
+    const long long off = x - pre[b];
+    const int g = (int)(off / npg);
+    const int j0 = (int)(off - (long long)g * npg);
+    const long long seg0 = pre[b] + (long long)g * npg;
+    const long long seg1 = seg0 + npg;
+    const long long xe = min(x_end, seg1);
+    const int j1 = j0 + (int)(xe - x);
+    const SeqPlan sp = make_plan(p.plan, b);
+    const int bg = b * Hkv + g;
+    const size_t head_off = (size_t)g * (kPage * kHeadDim);
+    const size_t page_stride = (size_t)Hkv * kPage * kHeadDim;
+
+    float qf[G][8];
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      const uint4 qv = *reinterpret_cast<const uint4*>(
+          p.q + ((size_t)b * p.hq + g * G + gg) * kHeadDim + 8 * li);
+      unpack8(qv, qf[gg]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qf[gg][e] *= p.scale_log2;
+    }
+    float m_run[VPL], l_run[VPL], acc[G][8];
+#pragma unroll
+    for (int u = 0; u < VPL; ++u) {
+      m_run[u] = -INFINITY;
+      l_run[u] = 0.f;
+    }
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[gg][e] = 0.f;
+
+    const int first = j0 + warp;
+    const int cnt = first < j1 ? (j1 - first + kWarps - 1) / kWarps : 0;
+
+    // lane 0 starts page n of this piece into stage (wcount + n) % kStages
+    auto issue = [&](int n) {
+      const int j = first + n * kWarps;
+      const PageRef r = page_ref(p.plan, sp, b, j);
+      uint64_t* bar = &wbar[(wcount + n) % kStages];
+      unsigned char* dst = wst + ((wcount + n) % kStages) * kStageBytes;
+      if (r.err == 0) {
+        const size_t src = (size_t)r.pb * page_stride + head_off;
+        mbar_arrive_expect_tx(bar, kStageBytes);
+        bulk_load(dst, p.k_cache + src, kPageBytes, bar, policy);
+        bulk_load(dst + kPageBytes, p.v_cache + src, kPageBytes, bar, policy);
+      } else {
+        report(p.status, r.err);
+        mbar_arrive(bar);
+      }
+    };
+
+    if (!dead && lane == 0)
+      for (int n = 0; n < min(cnt, kStages); ++n) issue(n);
+    __syncwarp();
+
+    for (int n = 0; n < cnt && !dead; ++n) {
+      const unsigned k = wcount + n;
+      const int stage = k % kStages;
+      const PageRef r = page_ref(p.plan, sp, b, first + n * kWarps);
+      if (!__all_sync(0xffffffffu, mbar_wait(&wbar[stage], (k / kStages) & 1u))) {
+        if (lane == 0) report(p.status, ODA_DEV_TIMEOUT);
+        // let the copies already started into the other stages land, then stop
+        for (int m = n + 1; m < min(cnt, n + kStages); ++m) {
+          const unsigned km = wcount + m;
+          mbar_wait(&wbar[km % kStages], (km / kStages) & 1u);
+        }
+        dead = true;
+        break;
+      }
+      if (r.err == 0) {
+        unsigned char* st = wst + stage * kStageBytes;
+        if (p.k_new != nullptr && r.lp == sp.t / kPage) {
+          // Commit: the step's K/V take slot t, in the cache and in this page's copy.
+          const int row = sp.t % kPage;
+          const bool isk = lane < 16;
+          const uint4 v = *reinterpret_cast<const uint4*>(
+              (isk ? p.k_new : p.v_new) + ((size_t)b * Hkv + g) * kHeadDim + 8 * li);
+          *reinterpret_cast<uint4*>(st + (isk ? 0 : kPageBytes) + row * kRowBytes + 16 * li) = v;
+          __nv_bfloat16* dst = (isk ? p.k_cache_w : p.v_cache_w) + (size_t)r.pb * page_stride +
+                               head_off + row * kHeadDim + 8 * li;
+          *reinterpret_cast<uint4*>(dst) = v;
+          fence_proxy_async_smem();  // this stage is refilled by a bulk copy later
+          __syncwarp();
+        }
+        page_step<G>(st, qf, m_run, l_run, acc, ps, sp, r.lp, lane, rows_vis);
+        ++pages_read;
+      }
+      __syncwarp();
+      if (lane == 0 && n + kStages < cnt) issue(n + kStages);
+      __syncwarp();
+    }
+    wcount += cnt;
+
+    // ---- merge the 8 half-warp states of this piece ----
+    float lsum[VPL];
+#pragma unroll
+    for (int u = 0; u < VPL; ++u) {
+      float v = l_run[u];
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      lsum[u] = v;
+    }
+    __syncthreads();  // every warp is done with its stages: reuse them as merge scratch
+    float* Mw = reinterpret_cast<float*>(stages);  // [2 * kWarps][G]
+    float* Lw = Mw + 2 * kWarps * G;               // [2 * kWarps][G]
+    float* Aw = Lw + 2 * kWarps * G;               // [2 * kWarps][G][128]
+    const int sidx = warp * 2 + half;
+    if (li < 2 && (G >= 2 || li == 0)) {
+#pragma unroll
+      for (int u = 0; u < VPL; ++u) {
+        const int gh = (G >= 2) ? ((li & 1) * (G / 2) + u) : 0;
+        Mw[sidx * G + gh] = m_run[u];
+        Lw[sidx * G + gh] = lsum[u];
+      }
+    }
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      float4* dst = reinterpret_cast<float4*>(Aw + (sidx * G + gg) * kHeadDim + 8 * li);
+      dst[0] = make_float4(acc[gg][0], acc[gg][1], acc[gg][2], acc[gg][3]);
+      dst[1] = make_float4(acc[gg][4], acc[gg][5], acc[gg][6], acc[gg][7]);
+    }
+    __syncthreads();
+    float o[G], l2[G];
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int s = 0; s < 2 * kWarps; ++s) M = fmaxf(M, Mw[s * G + gg]);
+      if (M == -INFINITY) {
+        o[gg] = 0.f;
+        l2[gg] = -INFINITY;
+      } else {
+        float L = 0.f, a = 0.f;
+#pragma unroll
+        for (int s = 0; s < 2 * kWarps; ++s) {
+          const float ms = Mw[s * G + gg];
+          const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+          L = fmaf(w, Lw[s * G + gg], L);
+          a = fmaf(w, Aw[(s * G + gg) * kHeadDim + tid], a);
+        }
+        o[gg] = a / L;
+        l2[gg] = M + log2f(L);
+      }
+    }
+
+    const int c_first = cta_of(seg0, T, Pe);
+    const int n_contrib = cta_of(seg1 - 1, T, Pe) - c_first + 1;
+    if (n_contrib == 1) {
+      write_final<G>(p, b, g, o, l2);
+    } else {
+      const size_t slot = (size_t)c + bg;
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        p.ws_o[(slot * G + gg) * kHeadDim + tid] = o[gg];
+        if (tid == 0) p.ws_lse[slot * G + gg] = l2[gg];
+      }
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) s_last = (atomicAdd(&p.ws_ticket[bg], 1u) == (unsigned)(n_contrib - 1));
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        const size_t s0 = (size_t)c_first + bg;
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg) {
+          float M = -INFINITY;
+          for (int s = 0; s < n_contrib; ++s) M = fmaxf(M, __ldcg(&p.ws_lse[(s0 + s) * G + gg]));
+          if (M == -INFINITY) {
+            o[gg] = 0.f;
+            l2[gg] = -INFINITY;
+          } else {
+            float L = 0.f, a = 0.f;
+            for (int s = 0; s < n_contrib; ++s) {
+              const float ls = __ldcg(&p.ws_lse[(s0 + s) * G + gg]);
+              const float w = (ls == -INFINITY) ? 0.f : exp2f(ls - M);
+              L += w;
+              a = fmaf(w, __ldcg(&p.ws_o[((s0 + s) * G + gg) * kHeadDim + tid]), a);
+            }
+            o[gg] = a / L;
+            l2[gg] = M + log2f(L);
+          }
+        }
+        write_final<G>(p, b, g, o, l2);
+        if (tid == 0) p.ws_ticket[bg] = 0u;  // leave the workspace zeroed
+      }
+    }
+    fence_proxy_async_smem();  // merge scratch is the next piece's stage memory
+    __syncthreads();
+    x = xe;
+  }
+
+  if (p.stats != nullptr) {
+    if (lane == 0) {
+      atomicAdd(&s_rows, (unsigned long long)rows_vis);
+      atomicAdd(&s_pages, (unsigned long long)pages_read);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      if (s_rows) atomicAdd(&p.stats[ODA_STAT_ROWS], s_rows);
+      if (s_pages) atomicAdd(&p.stats[ODA_STAT_PAGES], s_pages);
+    }
+  }
+}
+
+// Debug export of the same plan: mask[b][p] = 1 for every visible position p < max_tokens.
+__global__ void visible_mask_kernel(PlanArgs a, uint8_t* mask, int max_tokens, int* status) {
+  const int b = blockIdx.x;
+  uint8_t* row = mask + (size_t)b * max_tokens;
+  for (int i = threadIdx.x; i < max_tokens; i += blockDim.x) row[i] = 0;
+  __syncthreads();
+  const SeqPlan sp = make_plan(a, b);
+  if (sp.bad_len) report(status, ODA_DEV_BAD_LEN);
+  if (sp.bad_keep) report(status, ODA_DEV_BAD_KEEP_LIST);
+  if (sp.skip || sp.bad_len || sp.bad_keep) return;
+  for (int idx = threadIdx.x; idx < sp.npages * kPage; idx += blockDim.x) {
+    const int j = idx / kPage, r = idx % kPage;
+    const PageRef pr = page_ref(a, sp, b, j);
+    if (pr.err != 0) {
+      report(status, pr.err);
+      continue;
+    }
+    const int pos = pr.lp * kPage + r;
+    if (pos < max_tokens && row_visible(sp, pos)) row[pos] = 1;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------------------
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static size_t decode_smem_bytes(int G) {
+  return (size_t)kWarps * kStages * kStageBytes + (size_t)kWarps * kStages * sizeof(uint64_t) +
+         (size_t)kWarps * 18 * G * sizeof(float) + (size_t)(kMaxBatch + 1) * sizeof(int);
+}
+
+struct WsLayout {
+  size_t o_off, lse_off, ticket_off, total;
+};
+
+static WsLayout ws_layout(int batch, int hkv, int G, int grid) {
+  const size_t slots = (size_t)grid + (size_t)batch * hkv;
+  WsLayout w;
+  w.o_off = 0;
+  w.lse_off = align_up(slots * G * kHeadDim * sizeof(float), 256);
+  w.ticket_off = w.lse_off + align_up(slots * G * sizeof(float), 256);
+  w.total = w.ticket_off + align_up((size_t)batch * hkv * sizeof(unsigned), 256);
+  return w;
+}
+
+template <int G>
+static int prepare_decode_kernel(int device) {
+  static bool done[64] = {false};
+  if (device < 0 || device >= 64) return ODA_ERR_CUDA;
+  if (done[device]) return ODA_OK;
+  if (cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)decode_smem_bytes(G)) != cudaSuccess)
+    return ODA_ERR_CUDA;
+  done[device] = true;
+  return ODA_OK;
+}
+
+static int grid_size(const DeviceInfo& di) { return di.sms * kCtasPerSm; }
+
+int current_device_info(DeviceInfo* info) {
+  static DeviceInfo cache[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ODA_ERR_CUDA;
+  if (cache[dev].device != dev) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ODA_ERR_CUDA;
+    cache[dev].sms = sms;
+    cache[dev].device = dev;
+  }
+  *info = cache[dev];
+  return ODA_OK;
+}
+
+// Called before graph capture so that no attribute call happens while capturing.
+int prepare_decode_kernels() {
+  DeviceInfo di;
+  int rc = current_device_info(&di);
+  if (rc != ODA_OK) return rc;
+  if ((rc = prepare_decode_kernel<1>(di.device)) != ODA_OK) return rc;
+  if ((rc = prepare_decode_kernel<2>(di.device)) != ODA_OK) return rc;
+  return prepare_decode_kernel<4>(di.device);
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_kv(const oda_kv* kv) {
+  if (kv == nullptr) return ODA_ERR_INVALID_ARG;
+  if (kv->batch < 0 || kv->num_kv_heads < 1 || kv->max_blocks_per_seq < 1 || kv->num_blocks < 1)
+    return ODA_ERR_INVALID_ARG;
+  if (kv->head_dim != kHeadDim || kv->block_size != kPage) return ODA_ERR_UNSUPPORTED_SHAPE;
+  if (kv->batch > kMaxBatch) return ODA_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)kv->batch * kv->max_blocks_per_seq * kv->num_kv_heads >= (1ll << 31))
+    return ODA_ERR_UNSUPPORTED_SHAPE;
+  if (kv->batch > 0 && (kv->k_cache == nullptr || kv->v_cache == nullptr ||
+                        kv->block_table == nullptr || kv->seq_lens == nullptr))
+    return ODA_ERR_INVALID_ARG;
+  if (!aligned16(kv->k_cache) || !aligned16(kv->v_cache)) return ODA_ERR_INVALID_ARG;
+  return ODA_OK;
+}
+
+static int group_of(const oda_kv* kv, int hq, int* G) {
+  if (hq < 1 || hq % kv->num_kv_heads != 0) return ODA_ERR_UNSUPPORTED_SHAPE;
+  const int g = hq / kv->num_kv_heads;
+  if (g != 1 && g != 2 && g != 4) return ODA_ERR_UNSUPPORTED_SHAPE;
+  *G = g;
+  return ODA_OK;
+}
+
+static int launch_decode(const oda_kv* kv, int mode, const void* q, int hq, int sink,
+                         int window, float scale, const int32_t* gate,
+                         const int32_t* keep_blocks, const int32_t* keep_counts, int max_keep,
+                         const void* k_new, const void* v_new, void* out, int out_dtype,
+                         float* lse, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_kv(kv);
+  if (rc != ODA_OK) return rc;
+  int G = 0;
+  if ((rc = group_of(kv, hq, &G)) != ODA_OK) return rc;
+  if (out_dtype != ODA_F32 && out_dtype != ODA_BF16) return ODA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return ODA_ERR_INVALID_ARG;
+  if ((k_new == nullptr) != (v_new == nullptr)) return ODA_ERR_INVALID_ARG;
+  if (kv->batch == 0) return ODA_OK;
+  if (q == nullptr || out == nullptr || ws == nullptr) return ODA_ERR_INVALID_ARG;
+  if (!aligned16(q) || (k_new && (!aligned16(k_new) || !aligned16(v_new))))
+    return ODA_ERR_INVALID_ARG;
+  if (mode == ODA_MODE_KEEP && (keep_blocks == nullptr || keep_counts == nullptr || max_keep < 0 ||
+                                max_keep > kv->max_blocks_per_seq))
+    return ODA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if ((rc = current_device_info(&di)) != ODA_OK) return rc;
+  const int grid = grid_size(di);
+  const WsLayout wl = ws_layout(kv->batch, kv->num_kv_heads, G, grid);
+  if (ws_bytes < wl.total) return ODA_ERR_WORKSPACE_TOO_SMALL;
+
+  DecodeParams p;
+  p.plan.seq_lens = kv->seq_lens;
+  p.plan.block_table = kv->block_table;
+  p.plan.max_blocks = kv->max_blocks_per_seq;
+  p.plan.num_blocks = kv->num_blocks;
+  p.plan.mode = mode;
+  p.plan.sink = sink;
+  p.plan.window = window;
+  p.plan.gate = gate;
+  p.plan.keep_blocks = keep_blocks;
+  p.plan.keep_counts = keep_counts;
+  p.plan.max_keep = max_keep;
+  p.k_cache = static_cast<const __nv_bfloat16*>(kv->k_cache);
+  p.v_cache = static_cast<const __nv_bfloat16*>(kv->v_cache);
+  p.k_cache_w = static_cast<__nv_bfloat16*>(kv->k_cache);
+  p.v_cache_w = static_cast<__nv_bfloat16*>(kv->v_cache);
+  p.batch = kv->batch;
+  p.hkv = kv->num_kv_heads;
+  p.hq = hq;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = out;
+  p.out_bf16 = out_dtype == ODA_BF16;
+  p.lse = lse;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  p.ws_o = reinterpret_cast<float*>(w + wl.o_off);
+  p.ws_lse = reinterpret_cast<float*>(w + wl.lse_off);
+  p.ws_ticket = reinterpret_cast<unsigned*>(w + wl.ticket_off);
+  p.status = kv->dev_status;
+  p.stats = kv->stats;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t smem = decode_smem_bytes(G);
+  switch (G) {
+    case 1:
+      if ((rc = prepare_decode_kernel<1>(di.device)) != ODA_OK) return rc;
+      decode_kernel<1><<<grid, kThreads, smem, st>>>(p);
+      break;
+    case 2:
+      if ((rc = prepare_decode_kernel<2>(di.device)) != ODA_OK) return rc;
+      decode_kernel<2><<<grid, kThreads, smem, st>>>(p);
+      break;
+    default:
+      if ((rc = prepare_decode_kernel<4>(di.device)) != ODA_OK) return rc;
+      decode_kernel<4><<<grid, kThreads, smem, st>>>(p);
+      break;
+  }
+  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+}
+
+}  // namespace oda
+
+using namespace oda;
+
+extern "C" int oda_decode_workspace_size(int32_t batch, int32_t num_kv_heads,
+                                         int32_t num_q_heads, size_t* bytes) {
+  if (bytes == nullptr || batch < 0 || num_kv_heads < 1 || num_q_heads < 1)
+    return ODA_ERR_INVALID_ARG;
+  if (num_q_heads % num_kv_heads != 0) return ODA_ERR_UNSUPPORTED_SHAPE;
+  const int G = num_q_heads / num_kv_heads;
+  if (G > kMaxGroup) return ODA_ERR_UNSUPPORTED_SHAPE;
+  DeviceInfo di;
+  const int rc = current_device_info(&di);
+  if (rc != ODA_OK) return rc;
+  *bytes = ws_layout(batch, num_kv_heads, G, grid_size(di)).total;
+  return ODA_OK;
+}
+
+extern "C" int oda_decode_local(const oda_kv* kv, const void* q, int32_t num_q_heads,
+                                int32_t sink, int32_t window, float scale, const void* k_new,
+                                const void* v_new, void* out, int32_t out_dtype, float* lse,
+                                void* ws, size_t ws_bytes, void* stream) {
+  if (sink < 0 || window < 1) return ODA_ERR_INVALID_ARG;
+  return launch_decode(kv, ODA_MODE_LOCAL, q, num_q_heads, sink, window, scale, nullptr,
+                       nullptr, nullptr, 0, k_new, v_new, out, out_dtype, lse, ws, ws_bytes,
+                       stream);
+}
+
+extern "C" int oda_decode_full(const oda_kv* kv, const void* q, int32_t num_q_heads, float scale,
+                               const int32_t* gate, const void* k_new, const void* v_new,
+                               void* out, int32_t out_dtype, float* lse, void* ws,
+                               size_t ws_bytes, void* stream) {
+  return launch_decode(kv, ODA_MODE_FULL, q, num_q_heads, 0, 1, scale, gate, nullptr, nullptr,
+                       0, k_new, v_new, out, out_dtype, lse, ws, ws_bytes, stream);
+}
+
+extern "C" int oda_decode_blockmask(const oda_kv* kv, const void* q, int32_t num_q_heads,
+                                    float scale, const int32_t* keep_blocks,
+                                    const int32_t* keep_counts, int32_t max_keep, void* out,
+                                    int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  return launch_decode(kv, ODA_MODE_KEEP, q, num_q_heads, 0, 1, scale, nullptr, keep_blocks,
+                       keep_counts, max_keep, nullptr, nullptr, out, out_dtype, lse, ws,
+                       ws_bytes, stream);
+}
+
+extern "C" int oda_visible_mask(const oda_kv* kv, int32_t mode, int32_t sink, int32_t window,
+                                const int32_t* gate, const int32_t* keep_blocks,
+                                const int32_t* keep_counts, int32_t max_keep, uint8_t* mask,
+                                int32_t max_tokens, void* stream) {
+  int rc = check_kv(kv);
+  if (rc != ODA_OK) return rc;
+  if (mode != ODA_MODE_LOCAL && mode != ODA_MODE_FULL && mode != ODA_MODE_KEEP)
+    return ODA_ERR_INVALID_ARG;
+  if (mode == ODA_MODE_LOCAL && (sink < 0 || window < 1)) return ODA_ERR_INVALID_ARG;
+  if (mode == ODA_MODE_KEEP && (keep_blocks == nullptr || keep_counts == nullptr || max_keep < 0))
+    return ODA_ERR_INVALID_ARG;
+  if (max_tokens < 0 || (max_tokens > 0 && kv->batch > 0 && mask == nullptr))
+    return ODA_ERR_INVALID_ARG;
+  if (kv->batch == 0 || max_tokens == 0) return ODA_OK;
+  PlanArgs a;
+  a.seq_lens = kv->seq_lens;
+  a.block_table = kv->block_table;
+  a.max_blocks = kv->max_blocks_per_seq;
+  a.num_blocks = kv->num_blocks;
+  a.mode = mode;
+  a.sink = sink;
+  a.window = window;
+  a.gate = mode == ODA_MODE_FULL ? gate : nullptr;
+  a.keep_blocks = keep_blocks;
+  a.keep_counts = keep_counts;
+  a.max_keep = max_keep;
+  visible_mask_kernel<<<kv->batch, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      a, mask, max_tokens, kv->dev_status);
+  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+}

@@ -1,0 +1,206 @@
+// Step runtime: a whole ODA decode step as one CUDA graph ([ODA] 개발자 관점: Local, the FP32
+// recall head and the conditional Full recompute run in one GPU execution stream, e.g. CUDA
+// Graphs, so that routing needs no host synchronisation).
+//
+// Top-level graph:  [ev0] Local+commit x L  [ev1] recall  [ev2] IF(any gate) [ev3]
+// IF body:          Full+gated commit for every layer not marked local-only
+// The recall kernel sets the IF node's condition from the device; the condition resets to
+// 0 at every launch, so a step whose sequences are all Local skips the body entirely, and a
+// step with some gated sequences runs Full kernels that skip the ungated ones on-device.
+#include <stdlib.h>
+
+#include <new>
+
+#include "oda_common.cuh"
+
+namespace oda {
+int prepare_decode_kernels();
+}
+
+struct oda_step_graph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  cudaStream_t cap = nullptr;
+  cudaStream_t cap_body = nullptr;
+  cudaEvent_t placeholder[4] = {nullptr, nullptr, nullptr, nullptr};
+  cudaGraphNode_t ev_node[4] = {nullptr, nullptr, nullptr, nullptr};
+  bool timing = false;
+};
+
+namespace {
+
+void release(oda_step_graph* g) {
+  if (g == nullptr) return;
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  if (g->graph) cudaGraphDestroy(g->graph);
+  for (auto& e : g->placeholder)
+    if (e) cudaEventDestroy(e);
+  if (g->cap) cudaStreamDestroy(g->cap);
+  if (g->cap_body) cudaStreamDestroy(g->cap_body);
+  delete g;
+}
+
+// Record a timing event as a graph node and remember the node.
+int record_event_node(oda_step_graph* g, int i) {
+  if (cudaEventRecordWithFlags(g->placeholder[i], g->cap, cudaEventRecordExternal) != cudaSuccess)
+    return ODA_ERR_CUDA;
+  cudaStreamCaptureStatus st;
+  const cudaGraphNode_t* deps = nullptr;
+  size_t n = 0;
+  if (cudaStreamGetCaptureInfo(g->cap, &st, nullptr, nullptr, &deps, &n) != cudaSuccess || n != 1)
+    return ODA_ERR_CUDA;
+  g->ev_node[i] = deps[0];
+  return ODA_OK;
+}
+
+int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditionalHandle cond) {
+  const int L = d->num_layers;
+  int rc;
+  if (g->timing && (rc = record_event_node(g, 0)) != ODA_OK) return rc;
+  for (int l = 0; l < L; ++l) {
+    rc = oda_decode_local(&d->layers[l], d->q_local[l], d->num_q_heads, d->sink, d->window,
+                          d->scale, d->k_local[l], d->v_local[l], d->out[l], ODA_F32,
+                          d->lse ? d->lse[l] : nullptr, d->decode_ws, d->decode_ws_bytes, g->cap);
+    if (rc != ODA_OK) return rc;
+  }
+  if (g->timing && (rc = record_event_node(g, 1)) != ODA_OK) return rc;
+  const int hidden = d->num_q_heads * d->layers[0].head_dim;
+  rc = oda_recall_score(d->h_prev, d->emb, d->out[L - 1], ODA_F32, d->layers[0].batch, hidden,
+                        d->mlp, d->w1, d->b1, d->w2, d->b2, d->theta, d->q_out, d->gate_out,
+                        d->full_count, d->use_conditional ? (unsigned long long)cond : 0ull,
+                        d->recall_ws, d->recall_ws_bytes, g->cap);
+  if (rc != ODA_OK) return rc;
+  if (g->timing && (rc = record_event_node(g, 2)) != ODA_OK) return rc;
+
+  cudaStream_t full_stream = g->cap;
+  cudaGraph_t body = nullptr;
+  if (d->use_conditional) {
+    cudaStreamCaptureStatus st;
+    cudaGraph_t capg = nullptr;
+    const cudaGraphNode_t* deps = nullptr;
+    size_t n = 0;
+    if (cudaStreamGetCaptureInfo(g->cap, &st, nullptr, &capg, &deps, &n) != cudaSuccess)
+      return ODA_ERR_CUDA;
+    cudaGraphNodeParams cp = {};
+    cp.type = cudaGraphNodeTypeConditional;
+    cp.conditional.handle = cond;
+    cp.conditional.type = cudaGraphCondTypeIf;
+    cp.conditional.size = 1;
+    cudaGraphNode_t cnode;
+    if (cudaGraphAddNode(&cnode, capg, deps, n, &cp) != cudaSuccess) return ODA_ERR_CUDA;
+    body = cp.conditional.phGraph_out[0];
+    if (cudaStreamUpdateCaptureDependencies(g->cap, &cnode, 1, cudaStreamSetCaptureDependencies) !=
+        cudaSuccess)
+      return ODA_ERR_CUDA;
+    if (cudaStreamBeginCaptureToGraph(g->cap_body, body, nullptr, nullptr, 0,
+                                      cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+      return ODA_ERR_CUDA;
+    full_stream = g->cap_body;
+  }
+  for (int l = 0; l < L; ++l) {
+    if (d->local_only != nullptr && d->local_only[l]) continue;
+    rc = oda_decode_full(&d->layers[l], d->q_full[l], d->num_q_heads, d->scale, d->gate_out,
+                         d->k_full[l], d->v_full[l], d->out[l], ODA_F32,
+                         d->lse ? d->lse[l] : nullptr, d->decode_ws, d->decode_ws_bytes,
+                         full_stream);
+    if (rc != ODA_OK) break;
+  }
+  if (d->use_conditional) {
+    cudaGraph_t done = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(g->cap_body, &done);
+    if (rc != ODA_OK) return rc;
+    if (e != cudaSuccess) return ODA_ERR_CUDA;
+  }
+  if (rc != ODA_OK) return rc;
+  if (g->timing && (rc = record_event_node(g, 3)) != ODA_OK) return rc;
+  return ODA_OK;
+}
+
+int check_desc(const oda_step_desc* d) {
+  if (d == nullptr || d->num_layers < 1 || d->layers == nullptr) return ODA_ERR_INVALID_ARG;
+  if (!d->q_local || !d->k_local || !d->v_local || !d->q_full || !d->k_full || !d->v_full ||
+      !d->out)
+    return ODA_ERR_INVALID_ARG;
+  const oda_kv& k0 = d->layers[0];
+  for (int l = 1; l < d->num_layers; ++l) {
+    const oda_kv& k = d->layers[l];
+    if (k.batch != k0.batch || k.num_kv_heads != k0.num_kv_heads || k.seq_lens != k0.seq_lens ||
+        k.block_table != k0.block_table || k.max_blocks_per_seq != k0.max_blocks_per_seq)
+      return ODA_ERR_INVALID_ARG;
+  }
+  if (k0.batch < 1) return ODA_ERR_INVALID_ARG;
+  return ODA_OK;
+}
+
+}  // namespace
+
+extern "C" int oda_step_graph_create(const oda_step_desc* desc, void* stream,
+                                     oda_step_graph** graph) {
+  (void)stream;
+  if (graph == nullptr) return ODA_ERR_INVALID_ARG;
+  *graph = nullptr;
+  int rc = check_desc(desc);
+  if (rc != ODA_OK) return rc;
+  if ((rc = oda::prepare_decode_kernels()) != ODA_OK) return rc;
+  oda_step_graph* g = new (std::nothrow) oda_step_graph();
+  if (g == nullptr) return ODA_ERR_CUDA;
+  g->timing = desc->timing_events != 0;
+  if (cudaStreamCreateWithFlags(&g->cap, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&g->cap_body, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaGraphCreate(&g->graph, 0) != cudaSuccess) {
+    release(g);
+    return ODA_ERR_CUDA;
+  }
+  if (g->timing)
+    for (auto& e : g->placeholder)
+      if (cudaEventCreate(&e) != cudaSuccess) {
+        release(g);
+        return ODA_ERR_CUDA;
+      }
+  cudaGraphConditionalHandle cond = 0;
+  if (desc->use_conditional &&
+      cudaGraphConditionalHandleCreate(&cond, g->graph, 0, cudaGraphCondAssignDefault) !=
+          cudaSuccess) {
+    release(g);
+    return ODA_ERR_CUDA;
+  }
+  if (cudaStreamBeginCaptureToGraph(g->cap, g->graph, nullptr, nullptr, 0,
+                                    cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    release(g);
+    return ODA_ERR_CUDA;
+  }
+  rc = capture_step(desc, g, cond);
+  cudaGraph_t captured = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(g->cap, &captured);
+  if (rc == ODA_OK && e != cudaSuccess) rc = ODA_ERR_CUDA;
+  if (rc == ODA_OK && cudaGraphInstantiate(&g->exec, g->graph, 0) != cudaSuccess) rc = ODA_ERR_CUDA;
+  if (rc != ODA_OK) {
+    cudaGetLastError();
+    release(g);
+    return rc;
+  }
+  *graph = g;
+  return ODA_OK;
+}
+
+extern "C" int oda_step_graph_launch(oda_step_graph* graph, void* stream) {
+  if (graph == nullptr || graph->exec == nullptr) return ODA_ERR_INVALID_ARG;
+  return cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? ODA_OK
+             : ODA_ERR_CUDA;
+}
+
+extern "C" int oda_step_graph_set_events(oda_step_graph* graph, void* ev_start, void* ev_local,
+                                         void* ev_recall, void* ev_end) {
+  if (graph == nullptr || !graph->timing) return ODA_ERR_INVALID_ARG;
+  void* evs[4] = {ev_start, ev_local, ev_recall, ev_end};
+  for (int i = 0; i < 4; ++i) {
+    if (evs[i] == nullptr) return ODA_ERR_INVALID_ARG;
+    if (cudaGraphExecEventRecordNodeSetEvent(graph->exec, graph->ev_node[i],
+                                             static_cast<cudaEvent_t>(evs[i])) != cudaSuccess)
+      return ODA_ERR_CUDA;
+  }
+  return ODA_OK;
+}
+
+extern "C" void oda_step_graph_destroy(oda_step_graph* graph) { release(graph); }

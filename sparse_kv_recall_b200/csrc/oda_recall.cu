@@ -1,0 +1,232 @@
+// K4: recall head, gate, Full-rate counter and graph condition ([ODA] 접근 방법: the recall
+// head scores the step from h_{t-1}, E(x_t) and the current Local final hidden h^L_t, and
+// Full is recomputed iff q_t > theta; 개발자 관점: evaluated in FP32 on the GPU, inside the
+// same execution stream as Local and the conditional Full pass).
+//
+// q = w2 . GELU(W1^T x + b1) + b2 with x = [h_prev; emb; h_local] (3 * hidden rows of W1).
+// The 3*hidden x mlp weight matrix is split into kRows-row slabs x 64-column tiles, one CTA
+// each, so the whole GPU streams W1 once per call for every sequence of the batch. Per
+// column tile, the last slab CTA to finish (atomic ticket) sums the slabs' partial z in
+// fixed order and applies b1, GELU and w2; the last column tile then forms q, the gate, the
+// counter and the graph condition. Fixed orders make every result bitwise reproducible.
+#include <math.h>
+
+#include "oda_common.cuh"
+
+namespace oda {
+
+constexpr int kRThreads = 256;
+constexpr int kColTile = 64;
+constexpr int kRowGroups = kRThreads / kColTile;  // 4
+constexpr int kRows = 128;                        // rows of W1 per CTA
+constexpr int kBTile = 8;                         // sequences per pass over the slab
+
+struct RecallWs {
+  size_t z_off, q_off, ticket_off, total;
+  int slabs, tiles;
+};
+
+static size_t align_up_r(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static RecallWs recall_ws(int batch, int hidden, int mlp) {
+  RecallWs w;
+  w.slabs = (3 * hidden + kRows - 1) / kRows;
+  w.tiles = mlp / kColTile;
+  w.z_off = 0;
+  w.q_off = align_up_r((size_t)w.slabs * batch * mlp * sizeof(float), 256);
+  w.ticket_off = w.q_off + align_up_r((size_t)w.tiles * batch * sizeof(float), 256);
+  w.total = w.ticket_off + align_up_r((size_t)(w.tiles + 1) * sizeof(unsigned), 256);
+  return w;
+}
+
+__device__ __forceinline__ float gelu_erf(float z) {
+  return 0.5f * z * (1.f + erff(z * 0.70710678118654752f));
+}
+
+struct RecallParams {
+  const float* h_prev;
+  const float* emb;
+  const void* h_local;
+  int h_local_bf16;
+  int batch, hidden, mlp;
+  const float* w1;
+  const float* b1;
+  const float* w2;
+  float b2, theta;
+  float* q_out;
+  int32_t* gate_out;
+  unsigned long long* full_count;
+  cudaGraphConditionalHandle cond;
+  int use_cond;
+  float* z_part;      // [slabs][batch][mlp]
+  float* q_part;      // [tiles][batch]
+  unsigned* tickets;  // [tiles + 1]
+};
+
+__device__ __forceinline__ float x_at(const RecallParams& p, int b, int r) {
+  const int H = p.hidden;
+  if (r < H) return p.h_prev[(size_t)b * H + r];
+  if (r < 2 * H) return p.emb[(size_t)b * H + r - H];
+  const size_t i = (size_t)b * H + (r - 2 * H);
+  if (p.h_local_bf16)
+    return __bfloat162float(static_cast<const __nv_bfloat16*>(p.h_local)[i]);
+  return static_cast<const float*>(p.h_local)[i];
+}
+
+__global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p) {
+  __shared__ float xs[kBTile][kRows];
+  __shared__ float red[kRowGroups][kBTile][kColTile];
+  __shared__ int s_last;
+  __shared__ unsigned s_any, s_count;
+
+  const int tid = threadIdx.x;
+  const int rg = tid / kColTile, col = tid % kColTile;
+  const int slab = blockIdx.x, tile = blockIdx.y;
+  const int slabs = gridDim.x, tiles = gridDim.y;
+  const int R3 = 3 * p.hidden;
+  const int r0 = slab * kRows;
+  const int nrows = min(kRows, R3 - r0);
+  const int gcol = tile * kColTile + col;
+
+  // ---- partial z of this slab for every sequence ----
+  for (int b0 = 0; b0 < p.batch; b0 += kBTile) {
+    const int nb = min(kBTile, p.batch - b0);
+    for (int i = tid; i < kBTile * kRows; i += kRThreads) {
+      const int bb = i / kRows, r = i % kRows;
+      xs[bb][r] = (bb < nb && r < nrows) ? x_at(p, b0 + bb, r0 + r) : 0.f;
+    }
+    __syncthreads();
+    float acc[kBTile];
+#pragma unroll
+    for (int bb = 0; bb < kBTile; ++bb) acc[bb] = 0.f;
+    for (int r = rg; r < nrows; r += kRowGroups) {
+      const float w = p.w1[(size_t)(r0 + r) * p.mlp + gcol];
+#pragma unroll
+      for (int bb = 0; bb < kBTile; ++bb) acc[bb] = fmaf(xs[bb][r], w, acc[bb]);
+    }
+#pragma unroll
+    for (int bb = 0; bb < kBTile; ++bb) red[rg][bb][col] = acc[bb];
+    __syncthreads();
+    if (rg == 0) {
+      for (int bb = 0; bb < nb; ++bb) {
+        const float z = red[0][bb][col] + red[1][bb][col] + red[2][bb][col] + red[3][bb][col];
+        p.z_part[((size_t)slab * p.batch + b0 + bb) * p.mlp + gcol] = z;
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- last slab of this column tile: z, GELU, w2 ----
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&p.tickets[tile], 1u) == (unsigned)(slabs - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float* qsum = &red[0][0][0];  // [batch chunk of 4][64] reuse
+  for (int b0 = 0; b0 < p.batch; b0 += kRowGroups) {
+    const int b = b0 + rg;
+    float v = 0.f;
+    if (b < p.batch) {
+      float z = 0.f;
+      for (int s = 0; s < slabs; ++s) z += __ldcg(&p.z_part[((size_t)s * p.batch + b) * p.mlp + gcol]);
+      z += p.b1[gcol];
+      v = gelu_erf(z) * p.w2[gcol];
+    }
+    // sum over the 64 columns of this tile: two warps per sequence
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((tid & 31) == 0) qsum[tid >> 5] = v;
+    __syncthreads();
+    if (tid < kRowGroups && b0 + tid < p.batch)
+      p.q_part[(size_t)tile * p.batch + b0 + tid] = qsum[2 * tid] + qsum[2 * tid + 1];
+    __syncthreads();
+  }
+  if (tid == 0) p.tickets[tile] = 0u;
+
+  // ---- last column tile: q, gate, counter, condition ----
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    s_last = atomicAdd(&p.tickets[tiles], 1u) == (unsigned)(tiles - 1);
+    s_any = 0u;
+    s_count = 0u;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int b = tid; b < p.batch; b += kRThreads) {
+    float q = 0.f;
+    for (int t = 0; t < tiles; ++t) q += __ldcg(&p.q_part[(size_t)t * p.batch + b]);
+    q += p.b2;
+    const int gate = q > p.theta ? 1 : 0;
+    p.q_out[b] = q;
+    p.gate_out[b] = gate;
+    if (gate) {
+      atomicAdd(&s_count, 1u);
+      s_any = 1u;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    if (p.full_count != nullptr && s_count) {
+      atomicAdd(&p.full_count[0], (unsigned long long)s_count);
+      atomicAdd(&p.full_count[1], 1ull);
+    }
+    if (p.use_cond) cudaGraphSetConditional(p.cond, s_any ? 1u : 0u);
+    p.tickets[tiles] = 0u;
+  }
+}
+
+}  // namespace oda
+
+using namespace oda;
+
+extern "C" int oda_recall_workspace_size(int32_t batch, int32_t hidden, int32_t mlp,
+                                         size_t* bytes) {
+  if (bytes == nullptr || batch < 0 || hidden < 1 || mlp < kColTile || mlp % kColTile != 0)
+    return ODA_ERR_INVALID_ARG;
+  *bytes = recall_ws(batch, hidden, mlp).total;
+  return ODA_OK;
+}
+
+extern "C" int oda_recall_score(const float* h_prev, const float* emb, const void* h_local,
+                                int32_t h_local_dtype, int32_t batch, int32_t hidden,
+                                int32_t mlp, const float* w1, const float* b1, const float* w2,
+                                float b2, float theta, float* q_out, int32_t* gate_out,
+                                unsigned long long* full_count,
+                                unsigned long long graph_cond_handle, void* ws, size_t ws_bytes,
+                                void* stream) {
+  if (batch < 0 || hidden < 1 || mlp < kColTile || mlp % kColTile != 0) return ODA_ERR_INVALID_ARG;
+  if (h_local_dtype != ODA_F32 && h_local_dtype != ODA_BF16) return ODA_ERR_INVALID_ARG;
+  if (batch == 0) return ODA_OK;
+  if (!h_prev || !emb || !h_local || !w1 || !b1 || !w2 || !q_out || !gate_out || !ws)
+    return ODA_ERR_INVALID_ARG;
+  const RecallWs wl = recall_ws(batch, hidden, mlp);
+  if (ws_bytes < wl.total) return ODA_ERR_WORKSPACE_TOO_SMALL;
+  RecallParams p;
+  p.h_prev = h_prev;
+  p.emb = emb;
+  p.h_local = h_local;
+  p.h_local_bf16 = h_local_dtype == ODA_BF16;
+  p.batch = batch;
+  p.hidden = hidden;
+  p.mlp = mlp;
+  p.w1 = w1;
+  p.b1 = b1;
+  p.w2 = w2;
+  p.b2 = b2;
+  p.theta = theta;
+  p.q_out = q_out;
+  p.gate_out = gate_out;
+  p.full_count = full_count;
+  p.cond = static_cast<cudaGraphConditionalHandle>(graph_cond_handle);
+  p.use_cond = graph_cond_handle != 0ull;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  p.z_part = reinterpret_cast<float*>(w + wl.z_off);
+  p.q_part = reinterpret_cast<float*>(w + wl.q_off);
+  p.tickets = reinterpret_cast<unsigned*>(w + wl.ticket_off);
+  const dim3 grid(wl.slabs, wl.tiles);
+  recall_kernel<<<grid, kRThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+}

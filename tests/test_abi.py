@@ -1,0 +1,119 @@
+"""liboda builds, loads and exports every entry point include/oda.h declares; host-side
+argument checks return their codes without touching a GPU (no compute call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_kv_recall_b200 import build as B
+from sparse_kv_recall_b200 import oda
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "oda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return oda.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(oda_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "oda_decode_full" in names and len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(oda.exported_symbols()) == names
+
+
+def test_status_strings_and_version(lib):
+    for code, name in [(0, "ODA_OK"), (-1, "ODA_ERR_INVALID_ARG"), (-2, "ODA_ERR_UNSUPPORTED_SHAPE"),
+                       (-3, "ODA_ERR_WORKSPACE_TOO_SMALL"), (-4, "ODA_ERR_CUDA"),
+                       (-5, "ODA_ERR_NOT_IMPLEMENTED"), (1, "ODA_DEV_BAD_BLOCK"),
+                       (2, "ODA_DEV_BAD_LEN"), (3, "ODA_DEV_BAD_KEEP_LIST"), (4, "ODA_DEV_TIMEOUT")]:
+        assert oda.oda_status_string(code) == name
+    assert oda.oda_status_string(99) == "ODA_UNKNOWN_STATUS"
+    assert oda.oda_version() == 100
+
+
+def _kv(**kw):
+    base = dict(k_cache=0x10000, v_cache=0x20000, block_table=0x30000, seq_lens=0x40000, batch=2,
+                num_kv_heads=8, head_dim=128, block_size=16, max_blocks_per_seq=64, num_blocks=128,
+                dev_status=None, stats=None)
+    base.update(kw)
+    return oda.oda_kv(**base)
+
+
+def _local(lib, kv, hq=16, sink=4, window=256, scale=0.088, k_new=None, v_new=None, out=0x50000,
+           out_dtype=0, ws=0x60000, ws_bytes=1 << 40):
+    return lib.oda_decode_local(ctypes.byref(kv), 0x70000, hq, sink, window, scale, k_new, v_new, out,
+                                out_dtype, None, ws, ws_bytes, None)
+
+
+def test_decode_argument_checks(lib):
+    I, U = oda.ODA_ERR_INVALID_ARG, oda.ODA_ERR_UNSUPPORTED_SHAPE
+    assert lib.oda_decode_local(None, 0x70000, 16, 4, 256, 0.1, None, None, 0x50000, 0, None,
+                                0x60000, 1, None) == I
+    assert _local(lib, _kv(head_dim=64)) == U
+    assert _local(lib, _kv(block_size=32)) == U
+    assert _local(lib, _kv(), hq=12) == U                 # 12 query heads over 8 KV heads
+    assert _local(lib, _kv(), hq=64) == U                 # group of 8 is not built
+    assert _local(lib, _kv(), out_dtype=7) == I
+    assert _local(lib, _kv(), scale=0.0) == I
+    assert _local(lib, _kv(), scale=float("nan")) == I
+    assert _local(lib, _kv(), window=0) == I
+    assert _local(lib, _kv(), sink=-1) == I
+    assert _local(lib, _kv(), k_new=0x80000) == I         # k_new without v_new
+    assert _local(lib, _kv(k_cache=0x10008)) == I         # bulk copies need 16-byte alignment
+    assert _local(lib, _kv(batch=-1)) == I
+    assert _local(lib, _kv(batch=2000)) == U
+    assert _local(lib, _kv(batch=0)) == oda.ODA_OK         # nothing to do, nothing launched
+    kv = _kv()
+    assert lib.oda_decode_blockmask(ctypes.byref(kv), 0x70000, 16, 0.1, None, None, 4, 0x50000, 0,
+                                    None, 0x60000, 1, None) == I
+    assert lib.oda_decode_blockmask(ctypes.byref(kv), 0x70000, 16, 0.1, 0x1000, 0x2000, 65, 0x50000,
+                                    0, None, 0x60000, 1, None) == I   # max_keep > pages per seq
+    assert lib.oda_kv_append(ctypes.byref(_kv(num_kv_heads=40)), 0x1000, 0x2000, None, None) == U
+    assert lib.oda_kv_append(ctypes.byref(_kv()), None, 0x2000, None, None) == I
+    assert lib.oda_visible_mask(ctypes.byref(_kv()), 9, 4, 256, None, None, None, 0, 0x1000, 10,
+                                None) == I
+
+
+def test_workspace_queries(lib):
+    n = ctypes.c_size_t(0)
+    I = oda.ODA_ERR_INVALID_ARG
+    assert lib.oda_decode_workspace_size(1, 0, 16, ctypes.byref(n)) == I
+    assert lib.oda_decode_workspace_size(1, 8, 12, ctypes.byref(n)) == oda.ODA_ERR_UNSUPPORTED_SHAPE
+    assert lib.oda_recall_workspace_size(1, 2048, 100, ctypes.byref(n)) == I
+    sizes = []
+    for b in (1, 8, 16):
+        assert lib.oda_recall_workspace_size(b, 2048, 256, ctypes.byref(n)) == oda.ODA_OK
+        sizes.append(n.value)
+    assert 0 < sizes[0] < sizes[1] < sizes[2]
+    assert lib.oda_recall_score(0x1, 0x2, 0x3, 0, 1, 2048, 96, 0x4, 0x5, 0x6, 0.0, 0.0, 0x7, 0x8,
+                                None, 0, 0x9, 1 << 30, None) == I
+    assert lib.oda_recall_score(0x1, 0x2, 0x3, 0, 1, 2048, 256, 0x4, 0x5, 0x6, 0.0, 0.0, 0x7, 0x8,
+                                None, 0, 0x9, 16, None) == oda.ODA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_step_graph_argument_checks(lib):
+    h = ctypes.c_void_p(0)
+    assert lib.oda_step_graph_create(None, None, ctypes.byref(h)) == oda.ODA_ERR_INVALID_ARG
+    d = oda.oda_step_desc(num_layers=0)
+    assert lib.oda_step_graph_create(ctypes.byref(d), None, ctypes.byref(h)) == oda.ODA_ERR_INVALID_ARG
+    assert lib.oda_step_graph_launch(None, None) == oda.ODA_ERR_INVALID_ARG
+    assert lib.oda_step_graph_set_events(None, None, None, None, None) == oda.ODA_ERR_INVALID_ARG
+    lib.oda_step_graph_destroy(None)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(oda, "_lib", None)
+    monkeypatch.setattr(oda, "_LIB_PATH", str(tmp_path / "liboda.so"))
+    with pytest.raises(RuntimeError, match="liboda.so not found"):
+        oda.load()

@@ -1,0 +1,101 @@
+"""A whole ODA decode step (Local at every layer -> recall head -> conditional Full -> commit)
+as one graph launch, over several steps, against the oracle's step: per-layer outputs,
+recall scores, gates (ties within 1e-3 of theta excluded), committed K/V bits and the
+Full-call counter. Includes the 1-layer 4K workload in full (64 steps)."""
+import numpy as np
+import pytest
+import torch
+
+import oda_synth
+from oda_cases import Q_TOL, assert_attn_close
+from oracle import oda_oracle as O
+from sparse_kv_recall_b200 import build as B
+from sparse_kv_recall_b200 import oda
+from sparse_kv_recall_b200.engine import OdaEngine, fill_staging
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    B.build()
+    oda.load()
+
+
+def _logical(bits, bt, caps, hkv, d):
+    out = np.zeros((len(caps), hkv, max(caps), d), dtype=np.uint16)
+    for b, cap in enumerate(caps):
+        p = np.arange(cap)
+        out[b, :, :cap] = bits[bt[b, p // 16], :, p % 16, :].transpose(1, 0, 2)
+    return out
+
+
+def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02):
+    lay = oda_synth.make_layout(w, extra_tokens=steps + 2, device="cuda", lengths=lengths)
+    caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
+    rw = oda_synth.make_recall_weights(w, device="cuda", std=recall_std)
+    eng = OdaEngine([c[0] for c in caches], [c[1] for c in caches], lay.block_table,
+                    w.num_q_heads, (rw.w1, rw.b1, rw.w2, rw.b2), theta, sink=w.sink,
+                    window=w.window, use_conditional=use_conditional)
+    h0 = oda_synth.make_h0(w, device="cuda")
+    eng.set_h_prev(h0, 0)
+    bt = lay.block_table.cpu().numpy()
+    caps = lay.capacity
+    kh = [_logical(oda_synth.bf16_bits(c[0]), bt, caps, w.num_kv_heads, 128) for c in caches]
+    vh = [_logical(oda_synth.bf16_bits(c[1]), bt, caps, w.num_kv_heads, 128) for c in caches]
+    rec = (rw.w1.double().cpu().numpy(), rw.b1.double().cpu().numpy(),
+           rw.w2.double().cpu().numpy(), rw.b2)
+    dec = O.OdaDecoder(kh, vh, lengths, h0.double().cpu().numpy(), rec, sink=w.sink,
+                       window=w.window, theta=theta)
+    n_gated = 0
+    n_phases = 0
+    for i in range(steps):
+        si = oda_synth.make_step_inputs(w, i, device="cuda")
+        fill_staging(eng.v, si, [n + i + 1 for n in lengths])
+        eng.launch(i)
+        torch.cuda.synchronize()
+        assert int(eng.status.item()) == 0
+        outs = np.stack([eng.layer_out(i, l).cpu().numpy() for l in range(w.layers)])
+        q = eng.q_out.cpu().numpy()
+        gate = eng.gate.cpu().numpy().astype(bool)
+        inp = {k: [oda_synth.bf16_bits(x) for x in getattr(si, k)]
+               for k in ("q_local", "k_local", "v_local", "q_full", "k_full", "v_full")}
+        inp["emb"] = si.emb.double().cpu().numpy()
+        ref, _, rq, rg = dec.step(inp, gate_hint=gate)
+        assert np.abs(q - rq).max() <= Q_TOL, (i, q, rq)
+        sure = np.abs(rq - theta) >= Q_TOL
+        assert np.array_equal(gate[sure], rg[sure]), (i, gate, rg)
+        assert_attn_close(outs, ref, "step %d" % i)
+        n_gated += int(gate.sum())
+        n_phases += int(gate.any())
+    assert eng.full_count.cpu().tolist() == [n_gated, n_phases]
+    for l, (kc, vc) in enumerate(caches):                       # committed K/V, bit-exact
+        dk = _logical(oda_synth.bf16_bits(kc), bt, caps, w.num_kv_heads, 128)
+        dv = _logical(oda_synth.bf16_bits(vc), bt, caps, w.num_kv_heads, 128)
+        for b, n in enumerate(lengths):
+            assert np.array_equal(dk[b, :, :n + steps], dec.k[l][b, :, :n + steps])
+            assert np.array_equal(dv[b, :, :n + steps], dec.v[l][b, :, :n + steps])
+    eng.close()
+    return n_gated
+
+
+@pytest.mark.parametrize("use_conditional", [True, False])
+def test_step_graph_matches_oracle_ragged(use_conditional):
+    w = oda_synth.Workload(name="tiny", layers=3, batch=3, num_q_heads=16, num_kv_heads=8,
+                           prefill=300, steps=6, seed=77, sink=4, window=64)
+    n = _run_steps(w, [300, 37, 170], 6, theta=0.0, use_conditional=use_conditional)
+    assert 0 < n < 18                      # both paths exercised
+
+
+def test_step_graph_all_local_and_all_full():
+    w = oda_synth.Workload(name="tiny2", layers=2, batch=2, num_q_heads=32, num_kv_heads=8,
+                           prefill=500, steps=3, seed=78, sink=4, window=100)
+    assert _run_steps(w, [500, 129], 3, theta=float("inf")) == 0
+    assert _run_steps(w, [500, 129], 3, theta=-float("inf")) == 6
+
+
+def test_pr1_reference_workload_all_steps():
+    """1 layer, batch 1, 16 q / 8 KV heads, n = 4096, s = 4, w = 256, 64 steps, theta = 0."""
+    w = oda_synth.WORKLOADS["pr1-ref-4k"]
+    n = _run_steps(w, [w.prefill], w.steps, theta=w.theta)
+    assert 0 < n < w.steps
