@@ -52,13 +52,20 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["oda", "reference"], default="oda")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(oda_synth.WORKLOADS))
-    ap.add_argument("--calib-steps", type=int, default=64)
+    ap.add_argument("--calib-steps", type=int, default=512)
     ap.add_argument("--phase-steps", type=int, default=256)
     ap.add_argument("--kernel-reps", type=int, default=28)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--quick", action="store_true",
                     help="main timed region only (used for profiler launch lists)")
+    ap.add_argument("--no-conditional", action="store_true",
+                    help="Full kernels launch every step and skip ungated sequences on-device "
+                         "instead of sitting behind a graph IF node (ncu can list kernel nodes "
+                         "only of graphs without conditional nodes)")
+    ap.add_argument("--profile-kernel", choices=["full", "local", "recall"],
+                    help="one layer of the workload, the named kernel launched --steps times "
+                         "(a small case for ncu captures); prints nothing")
     return ap.parse_args()
 
 
@@ -195,7 +202,8 @@ def profiled_traffic(n_ctx_tokens_per_launch: float):
 class Setup:
     """Caches, recall head, engine and the resident pool of per-step inputs."""
 
-    def __init__(self, w, seed_offset: int, n_steps_total: int, theta: float, dev: str):
+    def __init__(self, w, seed_offset: int, n_steps_total: int, theta: float, dev: str,
+                 use_conditional: bool = True):
         from sparse_kv_recall_b200.engine import OdaEngine, StagingLayout, fill_staging
         self.w = oda_synth.scaled(w, seed=w.seed + 1000 * seed_offset)
         w = self.w
@@ -206,7 +214,7 @@ class Setup:
         self.recall = (rw.w1, rw.b1, rw.w2, rw.b2)
         self.eng = OdaEngine([c[0] for c in self.caches], [c[1] for c in self.caches],
                              self.layout.block_table, w.num_q_heads, self.recall, theta,
-                             sink=w.sink, window=w.window)
+                             sink=w.sink, window=w.window, use_conditional=use_conditional)
         self.eng.set_h_prev(oda_synth.make_h0(w, device=dev), 0)
         lay = StagingLayout(w.layers, w.batch, w.num_q_heads, w.num_kv_heads, w.hidden)
         self.slot = lay.nbytes
@@ -220,9 +228,9 @@ class Setup:
         self.eng.staging.copy_(self.pool[i], non_blocking=True)
 
 
-def launches_per_step(w, phases: int, steps: int) -> int:
+def launches_per_step(w, phases: int, steps: int, conditional: bool = True) -> int:
     """Kernels of this library launched by `steps` steps of which `phases` ran Full."""
-    return steps * (w.layers + 1) + phases * w.layers
+    return steps * (w.layers + 1) + (phases if conditional else steps) * w.layers
 
 
 def run_oda(args, dist: Dist):
@@ -241,7 +249,8 @@ def run_oda(args, dist: Dist):
     PH = 0 if args.quick else args.phase_steps
     E2E = 0 if (args.quick or args.no_e2e) else min(K, 256)
     total = C + W + K + PH + E2E
-    s = Setup(w, dist.rank, total, float("inf") if w.theta is None else w.theta, dev)
+    s = Setup(w, dist.rank, total, float("inf") if w.theta is None else w.theta, dev,
+              use_conditional=not args.no_conditional)
     eng = s.eng
     stream = torch.cuda.current_stream()
     step = 0
@@ -292,7 +301,7 @@ def run_oda(args, dist: Dist):
     rho = fc[0] / float(w.batch * K)
     kv_bytes = st[0] * ROW_BYTES
     page_bytes = st[1] * PAGE_BYTES
-    launches = launches_per_step(w, fc[1], K)
+    launches = launches_per_step(w, fc[1], K, not args.no_conditional)
     peak, peak_kind = measured_peak()
     result = {
         "metric": METRIC, "value": tokens / (ms / 1e3), "unit": UNIT, "n_gpus": dist.world,
@@ -303,7 +312,8 @@ def run_oda(args, dist: Dist):
                    "kv_heads": w.num_kv_heads, "head_dim": 128, "prefill": w.prefill,
                    "sink": w.sink, "window": w.window, "kv_dtype": "bf16",
                    "rho_target": w.target_rho, "rho_realised": rho, "theta": theta,
-                   "calibration_steps": C, "l2": "no flush: 15 GB KV stream per Full step >> 126 MB L2"
+                   "calibration_steps": C, "full_phase": "device early exit (no IF node)"
+                   if args.no_conditional else "graph IF node", "l2": "no flush: 15 GB KV stream per Full step >> 126 MB L2"
                    if w.name == DEFAULT_WORKLOAD else "no flush: KV working set > L2",
                    "parallelism": "replicas (dp%d, no collective)" % dist.world},
         "kv_stream": {"attended_bytes": kv_bytes, "gbs": kv_bytes / (ms_local / 1e3) / 1e9,
@@ -515,8 +525,47 @@ def run_reference(args, dist: Dist):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_profile_case(args):
+    """One layer of the workload (its KV pages still far larger than L2, a few GB at most),
+    one decode step's inputs, and the named kernel launched args.steps times."""
+    from sparse_kv_recall_b200 import build as B
+    from sparse_kv_recall_b200 import oda
+    B.build()
+    oda.load()
+    w = oda_synth.scaled(oda_synth.WORKLOADS[args.workload], layers=1)
+    dev = "cuda"
+    lengths = oda_synth.prefill_lengths(w)
+    lay = oda_synth.make_layout(w, extra_tokens=8, device=dev)
+    kc, vc = oda_synth.make_kv_cache(w, lay, 0, device=dev)
+    si = oda_synth.make_step_inputs(w, 0, device=dev)
+    seq = torch.tensor([n + 1 for n in lengths], dtype=torch.int32, device=dev)
+    kv = oda.make_kv(kc, vc, lay.block_table, seq)
+    ws = torch.zeros(oda.oda_decode_workspace_size(w.batch, w.num_kv_heads, w.num_q_heads),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float32, device=dev)
+    rw = oda_synth.make_recall_weights(w, device=dev)
+    rws = torch.zeros(oda.oda_recall_workspace_size(w.batch, w.hidden, w.mlp), dtype=torch.uint8,
+                      device=dev)
+    h = oda_synth.make_h0(w, device=dev)
+    qo = torch.empty(w.batch, dtype=torch.float32, device=dev)
+    go = torch.empty(w.batch, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(128)
+    for _ in range(args.steps):
+        if args.profile_kernel == "full":
+            oda.oda_decode_full(kv, si.q_full[0], scale, out, ws)
+        elif args.profile_kernel == "local":
+            oda.oda_decode_local(kv, si.q_local[0], w.sink, w.window, scale, out, ws)
+        else:
+            oda.oda_recall_score(h, si.emb, out.view(w.batch, -1), rw.w1, rw.b1, rw.w2, rw.b2,
+                                 0.0, qo, go, rws)
+    torch.cuda.synchronize()
+
+
 def main():
     args = parse_args()
+    if args.profile_kernel:
+        run_profile_case(args)
+        return
     dist = Dist(args.gpus)
     try:
         if args.impl == "reference":

@@ -179,21 +179,34 @@ def _bf16_normal(shape, g, device):
 
 
 def make_step_inputs(w: Workload, step: int, device="cpu") -> StepInputs:
+    """All per-layer q/k/v of one step, drawn in one N(0, 1) call and split into views."""
     B, Hq, Hkv, d = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim
+    nq, nk = B * Hq * d, B * Hkv * d
+    per_path = nq + 2 * nk
+    paths = [w.layers, max(w.layers - 1, 0)]          # Local: every layer; Full: layers >= 1
+    flat = _bf16_normal(((paths[0] + paths[1]) * per_path,), _gen(w.seed, _P_STEP, step,
+                                                                  device=device), device)
     cols = {k: [] for k in ("q_local", "k_local", "v_local", "q_full", "k_full", "v_full")}
+    off = 0
+
+    def take(n, shape):
+        nonlocal off
+        t = flat[off:off + n].view(shape)
+        off += n
+        return t
+
     for layer in range(w.layers):
-        g = _gen(w.seed, _P_STEP, step, layer, device=device)
-        ql = _bf16_normal((B, Hq, d), g, device)
-        kl = _bf16_normal((B, Hkv, d), g, device)
-        vl = _bf16_normal((B, Hkv, d), g, device)
+        cols["q_local"].append(take(nq, (B, Hq, d)))
+        cols["k_local"].append(take(nk, (B, Hkv, d)))
+        cols["v_local"].append(take(nk, (B, Hkv, d)))
+    for layer in range(w.layers):
         if layer == 0:
-            qf, kf, vf = ql, kl, vl
+            for k in ("q", "k", "v"):
+                cols[k + "_full"].append(cols[k + "_local"][0])
         else:
-            qf = _bf16_normal((B, Hq, d), g, device)
-            kf = _bf16_normal((B, Hkv, d), g, device)
-            vf = _bf16_normal((B, Hkv, d), g, device)
-        for k, v in zip(cols, (ql, kl, vl, qf, kf, vf)):
-            cols[k].append(v)
+            cols["q_full"].append(take(nq, (B, Hq, d)))
+            cols["k_full"].append(take(nk, (B, Hkv, d)))
+            cols["v_full"].append(take(nk, (B, Hkv, d)))
     ge = _gen(w.seed, _P_EMB, step, device=device)
     emb = torch.randn((B, w.hidden), generator=ge, device=device, dtype=torch.float32)
     return StepInputs(emb=emb, **cols)

@@ -2,10 +2,9 @@
 // path's current-position K/V joins the fully retained history). One warp per (sequence,
 // KV head): lanes 0-15 move the 256-byte K row, lanes 16-31 the V row, 16 bytes each.
 #include "oda_common.cuh"
+#include "oda_internal.h"
 
 namespace oda {
-
-int check_kv(const oda_kv* kv);
 
 __global__ void append_kernel(__nv_bfloat16* k_cache, __nv_bfloat16* v_cache,
                               const int32_t* block_table, const int32_t* seq_lens,

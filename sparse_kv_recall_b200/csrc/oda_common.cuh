@@ -110,6 +110,15 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return pol;
 }
 
+// ---- programmatic dependent launch -------------------------------------------------------
+// Wait until every prerequisite grid has completed and its writes are visible (returns at
+// once for a kernel launched without a programmatic dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel in the stream start its own pre-wait prologue.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- host side: per-device launch facts --------------------------------------------------
 struct DeviceInfo {
   int device = -1;

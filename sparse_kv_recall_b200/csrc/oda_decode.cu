@@ -18,6 +18,7 @@
 // (li % 2) * G / 2 + u.
 #include <math.h>
 
+#include "oda_internal.h"
 #include "oda_plan.cuh"
 
 namespace oda {
@@ -29,6 +30,8 @@ constexpr int kStageBytes = 2 * kPageBytes;
 constexpr int kCtasPerSm = 2;
 constexpr int kMaxBatch = 1024;
 constexpr int kMaxGroup = 4;
+constexpr int kMinShare = 8;            // units per CTA at least: bounds merge fan-in
+constexpr int kMergeChunk = 32;         // partials staged in shared memory at a time
 
 static_assert(kThreads == kHeadDim, "merge maps one thread per output dim");
 
@@ -51,6 +54,7 @@ struct DecodeParams {
   unsigned int* ws_ticket;     // [batch * hkv]
   int* status;
   unsigned long long* stats;
+  int wait_first;              // 1: the previous kernel may still write the gate: wait at once
 };
 
 // ---- reduce-scatter of C values over the 16 lanes of a half-warp ------------------------
@@ -173,6 +177,14 @@ __device__ __forceinline__ void write_final(const DecodeParams& p, int b, int g,
   }
 }
 
+// Arrive on a merge ticket: gpu-scope acquire-release add by one thread, after a CTA
+// barrier, publishes the CTA's partial and, for the last arrival, acquires all others.
+__device__ __forceinline__ unsigned ticket_arrive(unsigned* t) {
+  unsigned prev;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(t) : "memory");
+  return prev;
+}
+
 // CTA whose share contains flattened unit x (shares are [c*T/P, (c+1)*T/P), P <= T).
 __device__ __forceinline__ int cta_of(long long x, long long T, int P) {
   return (int)(((x + 1) * P - 1) / T);
@@ -195,6 +207,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   const int B = p.batch, Hkv = p.hkv;
   const int P = gridDim.x, c = blockIdx.x;
 
+  // Programmatic dependent launch: before griddep_wait this kernel only reads data that no
+  // kernel still in flight writes (lengths, page tables, keep lists, history pages) and fills
+  // shared memory; every global write and every read of q / k_new / v_new comes after it.
+  bool waited = false;
+  auto dep_wait = [&]() {
+    if (!waited) {
+      griddep_wait();
+      griddep_launch_dependents();
+      waited = true;
+    }
+  };
+  if (p.wait_first) dep_wait();
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[warp * kStages + s], 1);
@@ -214,11 +238,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     }
   }
   __syncthreads();
+  __shared__ int s_align;  // CTA-count granularity that keeps shares inside one (b, g)
   if (warp == 0) {  // inclusive scan of the per-sequence unit counts
     int carry = 0;
+    unsigned vmin = 0xffffffffu, vmax = 0u, active = 0u;
     for (int base = 0; base < B; base += 32) {
       const int i = base + lane;
       int v = i < B ? pre[i + 1] : 0;
+      const unsigned nz = (i < B && v > 0) ? (unsigned)v : 0u;
+      vmin = min(vmin, __reduce_min_sync(0xffffffffu, nz ? nz : 0xffffffffu));
+      vmax = max(vmax, __reduce_max_sync(0xffffffffu, nz));
+      active += __popc(__ballot_sync(0xffffffffu, nz != 0u));
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int n = __shfl_up_sync(0xffffffffu, v, o);
@@ -228,23 +258,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       if (i < B) pre[i + 1] = v;
       carry = __shfl_sync(0xffffffffu, v, 31);
     }
+    if (lane == 0) s_align = (active > 0 && vmin == vmax) ? (int)active * Hkv : 0;
   }
   __syncthreads();
   const long long T = pre[B];
-
-  // Sequences with nothing visible (bad length, empty keep list) but not gated off.
-  for (int bg = c; bg < B * Hkv; bg += P) {
-    const int b = bg / Hkv;
-    if (pre[b + 1] == pre[b] && !(p.plan.gate != nullptr && p.plan.gate[b] == 0)) {
-      float o[G], l2[G];
-#pragma unroll
-      for (int gg = 0; gg < G; ++gg) {
-        o[gg] = 0.f;
-        l2[gg] = -INFINITY;
-      }
-      write_final<G>(p, b, bg % Hkv, o, l2);
-    }
-  }
 
   const uint64_t policy = l2_evict_first_policy();
   unsigned char* wst = stages + warp * kStages * kStageBytes;
@@ -254,9 +271,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   bool dead = false;         // a bounded wait gave up: stop touching the ring
   unsigned rows_vis = 0, pages_read = 0;
 
-  // Shares go to the first Pe = min(P, T) CTAs only, so that every CTA holding a share has
-  // at least one unit and the CTAs that touch a (b, g) are exactly a contiguous index range.
-  const int Pe = (int)min((long long)P, T);
+  // Shares go to the first Pe <= min(P, ceil(T / kMinShare)) CTAs only, so that every CTA
+  // holding a share has at least one unit (and the CTAs that touch a (b, g) form a contiguous
+  // index range), and small launches do not fan a (b, g) out over more CTAs than they need.
+  int Pe = (int)min((long long)P, (T + kMinShare - 1) / kMinShare);
+  // When every non-empty sequence has the same page count, a multiple of (non-empty
+  // sequences x Hkv) CTAs makes every share fall inside one (b, g), so no CTA has to finish
+  // one piece before it can start streaming the next.
+  if (s_align > 0 && Pe >= s_align) Pe -= Pe % s_align;
   long long x = c < Pe ? (T * c) / Pe : 0;
   const long long x_end = c < Pe ? (T * (c + 1)) / Pe : 0;
   while (x < x_end) {
@@ -279,15 +301,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     const size_t head_off = (size_t)g * (kPage * kHeadDim);
     const size_t page_stride = (size_t)Hkv * kPage * kHeadDim;
 
-    float qf[G][8];
-#pragma unroll
-    for (int gg = 0; gg < G; ++gg) {
-      const uint4 qv = *reinterpret_cast<const uint4*>(
-          p.q + ((size_t)b * p.hq + g * G + gg) * kHeadDim + 8 * li);
-      unpack8(qv, qf[gg]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) qf[gg][e] *= p.scale_log2;
-    }
     float m_run[VPL], l_run[VPL], acc[G][8];
 #pragma unroll
     for (int u = 0; u < VPL; ++u) {
@@ -322,6 +335,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     if (!dead && lane == 0)
       for (int n = 0; n < min(cnt, kStages); ++n) issue(n);
     __syncwarp();
+    dep_wait();
+
+    float qf[G][8];
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      const uint4 qv = *reinterpret_cast<const uint4*>(
+          p.q + ((size_t)b * p.hq + g * G + gg) * kHeadDim + 8 * li);
+      unpack8(qv, qf[gg]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qf[gg][e] *= p.scale_log2;
+    }
 
     for (int n = 0; n < cnt && !dead; ++n) {
       const unsigned k = wcount + n;
@@ -425,29 +449,66 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
         p.ws_o[(slot * G + gg) * kHeadDim + tid] = o[gg];
         if (tid == 0) p.ws_lse[slot * G + gg] = l2[gg];
       }
-      __threadfence();
-      __syncthreads();
-      if (tid == 0) s_last = (atomicAdd(&p.ws_ticket[bg], 1u) == (unsigned)(n_contrib - 1));
-      __syncthreads();
+      __syncthreads();  // the CTA's partial is written; thread 0 publishes it (release)
+      if (tid == 0) s_last = ticket_arrive(&p.ws_ticket[bg]) == (unsigned)(n_contrib - 1);
+      __syncthreads();  // ... and the last CTA's thread 0 acquired everyone's partials
       if (s_last) {
-        __threadfence();
+        // Merge the n_contrib partials in fixed order: log-sums into shared memory (stage
+        // memory is free again), per-head max and weights by one warp per head, then every
+        // thread sums its dim over the partials with independent loads in flight.
         const size_t s0 = (size_t)c_first + bg;
+        float* sw = reinterpret_cast<float*>(stages);  // [n_contrib][G] log-sums -> weights
+        float* sml = sw + n_contrib * G;                // [G] max, [G] weight sum
+        float* so = sml + 2 * G + (4 - (n_contrib * G + 2 * G) % 4) % 4;  // float4-aligned
+        for (int i = tid; i < n_contrib * G; i += kThreads) sw[i] = __ldcg(&p.ws_lse[s0 * G + i]);
+        __syncthreads();
+        if (warp < G) {
+          float m = -INFINITY;
+          for (int s = lane; s < n_contrib; s += 32) m = fmaxf(m, sw[s * G + warp]);
+#pragma unroll
+          for (int o2 = 16; o2 >= 1; o2 >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o2));
+          float sum = 0.f;
+          for (int s = lane; s < n_contrib; s += 32) {
+            const float ls = sw[s * G + warp];
+            const float wgt = (ls == -INFINITY) ? 0.f : exp2f(ls - m);
+            sw[s * G + warp] = wgt;
+            sum += wgt;
+          }
+#pragma unroll
+          for (int o2 = 16; o2 >= 1; o2 >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o2);
+          if (lane == 0) {
+            sml[warp] = m;
+            sml[G + warp] = sum;
+          }
+        }
+        float a[G];
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg) a[gg] = 0.f;
+        // Partials are staged through shared memory kMergeChunk at a time with independent
+        // 16-byte loads, then summed in fixed order by the thread that owns each dim.
+        const float4* src = reinterpret_cast<const float4*>(p.ws_o + s0 * G * kHeadDim);
+        float4* dst4 = reinterpret_cast<float4*>(so);
+        for (int s_lo = 0; s_lo < n_contrib; s_lo += kMergeChunk) {
+          const int ns = min(kMergeChunk, n_contrib - s_lo);
+          const int n4 = ns * G * kHeadDim / 4;
+          const float4* src_c = src + (size_t)s_lo * G * kHeadDim / 4;
+          __syncthreads();
+#pragma unroll 8
+          for (int i = tid; i < n4; i += kThreads) dst4[i] = __ldcg(src_c + i);
+          __syncthreads();
+          for (int s = 0; s < ns; ++s)
+#pragma unroll
+            for (int gg = 0; gg < G; ++gg)
+              a[gg] = fmaf(sw[(s_lo + s) * G + gg], so[(s * G + gg) * kHeadDim + tid], a[gg]);
+        }
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) {
-          float M = -INFINITY;
-          for (int s = 0; s < n_contrib; ++s) M = fmaxf(M, __ldcg(&p.ws_lse[(s0 + s) * G + gg]));
+          const float M = sml[gg], L = sml[G + gg];
           if (M == -INFINITY) {
             o[gg] = 0.f;
             l2[gg] = -INFINITY;
           } else {
-            float L = 0.f, a = 0.f;
-            for (int s = 0; s < n_contrib; ++s) {
-              const float ls = __ldcg(&p.ws_lse[(s0 + s) * G + gg]);
-              const float w = (ls == -INFINITY) ? 0.f : exp2f(ls - M);
-              L += w;
-              a = fmaf(w, __ldcg(&p.ws_o[((s0 + s) * G + gg) * kHeadDim + tid]), a);
-            }
-            o[gg] = a / L;
+            o[gg] = a[gg] / L;
             l2[gg] = M + log2f(L);
           }
         }
@@ -458,6 +519,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     fence_proxy_async_smem();  // merge scratch is the next piece's stage memory
     __syncthreads();
     x = xe;
+  }
+
+  // Sequences with nothing visible (bad length, empty keep list) but not gated off.
+  dep_wait();
+  for (int bg = c; bg < B * Hkv; bg += P) {
+    const int b = bg / Hkv;
+    if (pre[b + 1] == pre[b] && !(p.plan.gate != nullptr && p.plan.gate[b] == 0)) {
+      float o[G], l2[G];
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        o[gg] = 0.f;
+        l2[gg] = -INFINITY;
+      }
+      write_final<G>(p, b, bg % Hkv, o, l2);
+    }
   }
 
   if (p.stats != nullptr) {
@@ -583,11 +659,27 @@ static int group_of(const oda_kv* kv, int hq, int* G) {
   return ODA_OK;
 }
 
-static int launch_decode(const oda_kv* kv, int mode, const void* q, int hq, int sink,
-                         int window, float scale, const int32_t* gate,
-                         const int32_t* keep_blocks, const int32_t* keep_counts, int max_keep,
-                         const void* k_new, const void* v_new, void* out, int out_dtype,
-                         float* lse, void* ws, size_t ws_bytes, void* stream) {
+template <int G>
+static cudaError_t launch_decode_kernel(const DecodeParams& p, int grid, size_t smem,
+                                        cudaStream_t st, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<G>, p);
+}
+
+int launch_decode(const oda_kv* kv, int mode, const void* q, int hq, int sink, int window,
+                  float scale, const int32_t* gate, const int32_t* keep_blocks,
+                  const int32_t* keep_counts, int max_keep, const void* k_new,
+                  const void* v_new, void* out, int out_dtype, float* lse, void* ws,
+                  size_t ws_bytes, void* stream, int pdl, int wait_first) {
   int rc = check_kv(kv);
   if (rc != ODA_OK) return rc;
   int G = 0;
@@ -640,29 +732,45 @@ static int launch_decode(const oda_kv* kv, int mode, const void* q, int hq, int 
   p.ws_ticket = reinterpret_cast<unsigned*>(w + wl.ticket_off);
   p.status = kv->dev_status;
   p.stats = kv->stats;
+  p.wait_first = wait_first;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t smem = decode_smem_bytes(G);
+  cudaError_t e;
   switch (G) {
     case 1:
       if ((rc = prepare_decode_kernel<1>(di.device)) != ODA_OK) return rc;
-      decode_kernel<1><<<grid, kThreads, smem, st>>>(p);
+      e = launch_decode_kernel<1>(p, grid, smem, st, pdl != 0);
       break;
     case 2:
       if ((rc = prepare_decode_kernel<2>(di.device)) != ODA_OK) return rc;
-      decode_kernel<2><<<grid, kThreads, smem, st>>>(p);
+      e = launch_decode_kernel<2>(p, grid, smem, st, pdl != 0);
       break;
     default:
       if ((rc = prepare_decode_kernel<4>(di.device)) != ODA_OK) return rc;
-      decode_kernel<4><<<grid, kThreads, smem, st>>>(p);
+      e = launch_decode_kernel<4>(p, grid, smem, st, pdl != 0);
       break;
   }
-  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  return e == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
 }
 
 }  // namespace oda
 
 using namespace oda;
+
+namespace oda {
+int decode_ws_layout(int batch, int hkv, int hq, size_t* total, size_t* ticket_off) {
+  if (batch < 0 || hkv < 1 || hq < 1 || hq % hkv != 0 || hq / hkv > kMaxGroup)
+    return ODA_ERR_UNSUPPORTED_SHAPE;
+  DeviceInfo di;
+  const int rc = current_device_info(&di);
+  if (rc != ODA_OK) return rc;
+  const WsLayout wl = ws_layout(batch, hkv, hq / hkv, grid_size(di));
+  *total = wl.total;
+  *ticket_off = wl.ticket_off;
+  return ODA_OK;
+}
+}  // namespace oda
 
 extern "C" int oda_decode_workspace_size(int32_t batch, int32_t num_kv_heads,
                                          int32_t num_q_heads, size_t* bytes) {
@@ -685,7 +793,7 @@ extern "C" int oda_decode_local(const oda_kv* kv, const void* q, int32_t num_q_h
   if (sink < 0 || window < 1) return ODA_ERR_INVALID_ARG;
   return launch_decode(kv, ODA_MODE_LOCAL, q, num_q_heads, sink, window, scale, nullptr,
                        nullptr, nullptr, 0, k_new, v_new, out, out_dtype, lse, ws, ws_bytes,
-                       stream);
+                       stream, 0, 0);
 }
 
 extern "C" int oda_decode_full(const oda_kv* kv, const void* q, int32_t num_q_heads, float scale,
@@ -693,7 +801,7 @@ extern "C" int oda_decode_full(const oda_kv* kv, const void* q, int32_t num_q_he
                                void* out, int32_t out_dtype, float* lse, void* ws,
                                size_t ws_bytes, void* stream) {
   return launch_decode(kv, ODA_MODE_FULL, q, num_q_heads, 0, 1, scale, gate, nullptr, nullptr,
-                       0, k_new, v_new, out, out_dtype, lse, ws, ws_bytes, stream);
+                       0, k_new, v_new, out, out_dtype, lse, ws, ws_bytes, stream, 0, 0);
 }
 
 extern "C" int oda_decode_blockmask(const oda_kv* kv, const void* q, int32_t num_q_heads,
@@ -703,7 +811,7 @@ extern "C" int oda_decode_blockmask(const oda_kv* kv, const void* q, int32_t num
                                     void* stream) {
   return launch_decode(kv, ODA_MODE_KEEP, q, num_q_heads, 0, 1, scale, nullptr, keep_blocks,
                        keep_counts, max_keep, nullptr, nullptr, out, out_dtype, lse, ws,
-                       ws_bytes, stream);
+                       ws_bytes, stream, 0, 0);
 }
 
 extern "C" int oda_visible_mask(const oda_kv* kv, int32_t mode, int32_t sink, int32_t window,
@@ -736,3 +844,4 @@ extern "C" int oda_visible_mask(const oda_kv* kv, int32_t mode, int32_t sink, in
       a, mask, max_tokens, kv->dev_status);
   return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
 }
+

@@ -12,10 +12,7 @@
 #include <new>
 
 #include "oda_common.cuh"
-
-namespace oda {
-int prepare_decode_kernels();
-}
+#include "oda_internal.h"
 
 struct oda_step_graph {
   cudaGraph_t graph = nullptr;
@@ -57,18 +54,25 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
   const int L = d->num_layers;
   int rc;
   if (g->timing && (rc = record_event_node(g, 0)) != ODA_OK) return rc;
+  // Programmatic dependent launch between consecutive kernels: each Local layer after the
+  // first, the recall head after the last Local layer and each Full layer after the first
+  // may start while its predecessor finishes (see the kernels for what they do before
+  // waiting). Kernels next to a timing-event node keep ordinary launches.
   for (int l = 0; l < L; ++l) {
-    rc = oda_decode_local(&d->layers[l], d->q_local[l], d->num_q_heads, d->sink, d->window,
-                          d->scale, d->k_local[l], d->v_local[l], d->out[l], ODA_F32,
-                          d->lse ? d->lse[l] : nullptr, d->decode_ws, d->decode_ws_bytes, g->cap);
+    if (d->sink < 0 || d->window < 1) return ODA_ERR_INVALID_ARG;
+    rc = oda::launch_decode(&d->layers[l], ODA_MODE_LOCAL, d->q_local[l], d->num_q_heads,
+                            d->sink, d->window, d->scale, nullptr, nullptr, nullptr, 0,
+                            d->k_local[l], d->v_local[l], d->out[l], ODA_F32,
+                            d->lse ? d->lse[l] : nullptr, d->decode_ws, d->decode_ws_bytes,
+                            g->cap, l > 0 ? 1 : 0, 0);
     if (rc != ODA_OK) return rc;
   }
   if (g->timing && (rc = record_event_node(g, 1)) != ODA_OK) return rc;
   const int hidden = d->num_q_heads * d->layers[0].head_dim;
-  rc = oda_recall_score(d->h_prev, d->emb, d->out[L - 1], ODA_F32, d->layers[0].batch, hidden,
-                        d->mlp, d->w1, d->b1, d->w2, d->b2, d->theta, d->q_out, d->gate_out,
-                        d->full_count, d->use_conditional ? (unsigned long long)cond : 0ull,
-                        d->recall_ws, d->recall_ws_bytes, g->cap);
+  rc = oda::launch_recall(d->h_prev, d->emb, d->out[L - 1], ODA_F32, d->layers[0].batch, hidden,
+                          d->mlp, d->w1, d->b1, d->w2, d->b2, d->theta, d->q_out, d->gate_out,
+                          d->full_count, d->use_conditional ? (unsigned long long)cond : 0ull,
+                          d->recall_ws, d->recall_ws_bytes, g->cap, g->timing ? 0 : 1);
   if (rc != ODA_OK) return rc;
   if (g->timing && (rc = record_event_node(g, 2)) != ODA_OK) return rc;
 
@@ -97,12 +101,21 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
       return ODA_ERR_CUDA;
     full_stream = g->cap_body;
   }
+  bool first_full = true;
   for (int l = 0; l < L; ++l) {
     if (d->local_only != nullptr && d->local_only[l]) continue;
-    rc = oda_decode_full(&d->layers[l], d->q_full[l], d->num_q_heads, d->scale, d->gate_out,
-                         d->k_full[l], d->v_full[l], d->out[l], ODA_F32,
-                         d->lse ? d->lse[l] : nullptr, d->decode_ws, d->decode_ws_bytes,
-                         full_stream);
+    // The first Full kernel reads the gate the recall head just wrote: inside the IF body it
+    // is the body's first node; without the IF node it waits for the recall head at once.
+    int pdl = 1, wait_first = 0;
+    if (first_full) {
+      pdl = (!d->use_conditional && !g->timing) ? 1 : 0;
+      wait_first = 1;
+    }
+    rc = oda::launch_decode(&d->layers[l], ODA_MODE_FULL, d->q_full[l], d->num_q_heads, 0, 1,
+                            d->scale, d->gate_out, nullptr, nullptr, 0, d->k_full[l],
+                            d->v_full[l], d->out[l], ODA_F32, d->lse ? d->lse[l] : nullptr,
+                            d->decode_ws, d->decode_ws_bytes, full_stream, pdl, wait_first);
+    first_full = false;
     if (rc != ODA_OK) break;
   }
   if (d->use_conditional) {

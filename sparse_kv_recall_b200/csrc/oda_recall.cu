@@ -12,6 +12,7 @@
 #include <math.h>
 
 #include "oda_common.cuh"
+#include "oda_internal.h"
 
 namespace oda {
 
@@ -19,6 +20,7 @@ constexpr int kRThreads = 256;
 constexpr int kColTile = 64;
 constexpr int kRowGroups = kRThreads / kColTile;  // 4
 constexpr int kRows = 128;                        // rows of W1 per CTA
+constexpr int kRowsPerThread = kRows / kRowGroups;
 constexpr int kBTile = 8;                         // sequences per pass over the slab
 
 struct RecallWs {
@@ -76,6 +78,7 @@ __device__ __forceinline__ float x_at(const RecallParams& p, int b, int r) {
 __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p) {
   __shared__ float xs[kBTile][kRows];
   __shared__ float red[kRowGroups][kBTile][kColTile];
+  __shared__ float qs[kBTile][2];
   __shared__ int s_last;
   __shared__ unsigned s_any, s_count;
 
@@ -83,10 +86,21 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
   const int rg = tid / kColTile, col = tid % kColTile;
   const int slab = blockIdx.x, tile = blockIdx.y;
   const int slabs = gridDim.x, tiles = gridDim.y;
-  const int R3 = 3 * p.hidden;
   const int r0 = slab * kRows;
-  const int nrows = min(kRows, R3 - r0);
+  const int nrows = min(kRows, 3 * p.hidden - r0);
   const int gcol = tile * kColTile + col;
+
+  // Slabs that read only h_prev and emb rows may run while the previous kernel (the last
+  // Local layer, which writes h_local) finishes; the others wait for it first.
+  if (r0 + nrows > 2 * p.hidden) griddep_wait();
+  griddep_launch_dependents();
+
+  float wv[kRowsPerThread];  // this thread's W1 column over its rows, all loads in flight
+#pragma unroll
+  for (int i = 0; i < kRowsPerThread; ++i) {
+    const int r = rg + i * kRowGroups;
+    wv[i] = r < nrows ? __ldg(&p.w1[(size_t)(r0 + r) * p.mlp + gcol]) : 0.f;
+  }
 
   // ---- partial z of this slab for every sequence ----
   for (int b0 = 0; b0 < p.batch; b0 += kBTile) {
@@ -99,10 +113,11 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
     float acc[kBTile];
 #pragma unroll
     for (int bb = 0; bb < kBTile; ++bb) acc[bb] = 0.f;
-    for (int r = rg; r < nrows; r += kRowGroups) {
-      const float w = p.w1[(size_t)(r0 + r) * p.mlp + gcol];
 #pragma unroll
-      for (int bb = 0; bb < kBTile; ++bb) acc[bb] = fmaf(xs[bb][r], w, acc[bb]);
+    for (int i = 0; i < kRowsPerThread; ++i) {
+      const int r = rg + i * kRowGroups;
+#pragma unroll
+      for (int bb = 0; bb < kBTile; ++bb) acc[bb] = fmaf(xs[bb][r], wv[i], acc[bb]);
     }
 #pragma unroll
     for (int bb = 0; bb < kBTile; ++bb) red[rg][bb][col] = acc[bb];
@@ -116,35 +131,44 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
     __syncthreads();
   }
 
-  // ---- last slab of this column tile: z, GELU, w2 ----
+  // ---- last slab of this column tile: z, GELU, w2 (summed over the tile's columns) ----
   __threadfence();
   __syncthreads();
   if (tid == 0) s_last = atomicAdd(&p.tickets[tile], 1u) == (unsigned)(slabs - 1);
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  float* qsum = &red[0][0][0];  // [batch chunk of 4][64] reuse
-  for (int b0 = 0; b0 < p.batch; b0 += kRowGroups) {
-    const int b = b0 + rg;
-    float v = 0.f;
-    if (b < p.batch) {
-      float z = 0.f;
-      for (int s = 0; s < slabs; ++s) z += __ldcg(&p.z_part[((size_t)s * p.batch + b) * p.mlp + gcol]);
-      z += p.b1[gcol];
-      v = gelu_erf(z) * p.w2[gcol];
-    }
-    // sum over the 64 columns of this tile: two warps per sequence
+  for (int b0 = 0; b0 < p.batch; b0 += kBTile) {
+    const int nb = min(kBTile, p.batch - b0);
+    float zz[kBTile];
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if ((tid & 31) == 0) qsum[tid >> 5] = v;
+    for (int bb = 0; bb < kBTile; ++bb) zz[bb] = 0.f;
+#pragma unroll 4
+    for (int sl = rg; sl < slabs; sl += kRowGroups) {
+#pragma unroll
+      for (int bb = 0; bb < kBTile; ++bb)
+        if (bb < nb) zz[bb] += __ldcg(&p.z_part[((size_t)sl * p.batch + b0 + bb) * p.mlp + gcol]);
+    }
+#pragma unroll
+    for (int bb = 0; bb < kBTile; ++bb) red[rg][bb][col] = zz[bb];
     __syncthreads();
-    if (tid < kRowGroups && b0 + tid < p.batch)
-      p.q_part[(size_t)tile * p.batch + b0 + tid] = qsum[2 * tid] + qsum[2 * tid + 1];
+    if (tid < kColTile) {  // warps 0 and 1: one column each
+      for (int bb = 0; bb < nb; ++bb) {
+        const float z = red[0][bb][col] + red[1][bb][col] + red[2][bb][col] + red[3][bb][col] +
+                        p.b1[gcol];
+        float v = gelu_erf(z) * p.w2[gcol];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if ((tid & 31) == 0) qs[bb][tid >> 5] = v;
+      }
+    }
+    __syncthreads();
+    if (tid < nb) p.q_part[(size_t)tile * p.batch + b0 + tid] = qs[tid][0] + qs[tid][1];
     __syncthreads();
   }
   if (tid == 0) p.tickets[tile] = 0u;
 
-  // ---- last column tile: q, gate, counter, condition ----
+  // ---- last column tile: q, gate, counters, condition ----
   __threadfence();
   __syncthreads();
   if (tid == 0) {
@@ -178,25 +202,11 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
   }
 }
 
-}  // namespace oda
-
-using namespace oda;
-
-extern "C" int oda_recall_workspace_size(int32_t batch, int32_t hidden, int32_t mlp,
-                                         size_t* bytes) {
-  if (bytes == nullptr || batch < 0 || hidden < 1 || mlp < kColTile || mlp % kColTile != 0)
-    return ODA_ERR_INVALID_ARG;
-  *bytes = recall_ws(batch, hidden, mlp).total;
-  return ODA_OK;
-}
-
-extern "C" int oda_recall_score(const float* h_prev, const float* emb, const void* h_local,
-                                int32_t h_local_dtype, int32_t batch, int32_t hidden,
-                                int32_t mlp, const float* w1, const float* b1, const float* w2,
-                                float b2, float theta, float* q_out, int32_t* gate_out,
-                                unsigned long long* full_count,
-                                unsigned long long graph_cond_handle, void* ws, size_t ws_bytes,
-                                void* stream) {
+int launch_recall(const float* h_prev, const float* emb, const void* h_local, int h_local_dtype,
+                  int batch, int hidden, int mlp, const float* w1, const float* b1,
+                  const float* w2, float b2, float theta, float* q_out, int32_t* gate_out,
+                  unsigned long long* full_count, unsigned long long graph_cond_handle,
+                  void* ws, size_t ws_bytes, void* stream, int pdl) {
   if (batch < 0 || hidden < 1 || mlp < kColTile || mlp % kColTile != 0) return ODA_ERR_INVALID_ARG;
   if (h_local_dtype != ODA_F32 && h_local_dtype != ODA_BF16) return ODA_ERR_INVALID_ARG;
   if (batch == 0) return ODA_OK;
@@ -226,7 +236,38 @@ extern "C" int oda_recall_score(const float* h_prev, const float* emb, const voi
   p.z_part = reinterpret_cast<float*>(w + wl.z_off);
   p.q_part = reinterpret_cast<float*>(w + wl.q_off);
   p.tickets = reinterpret_cast<unsigned*>(w + wl.ticket_off);
-  const dim3 grid(wl.slabs, wl.tiles);
-  recall_kernel<<<grid, kRThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
-  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(wl.slabs, wl.tiles);
+  cfg.blockDim = dim3(kRThreads);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, recall_kernel, p) == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+}
+
+}  // namespace oda
+
+using namespace oda;
+
+extern "C" int oda_recall_workspace_size(int32_t batch, int32_t hidden, int32_t mlp,
+                                         size_t* bytes) {
+  if (bytes == nullptr || batch < 0 || hidden < 1 || mlp < kColTile || mlp % kColTile != 0)
+    return ODA_ERR_INVALID_ARG;
+  *bytes = recall_ws(batch, hidden, mlp).total;
+  return ODA_OK;
+}
+
+extern "C" int oda_recall_score(const float* h_prev, const float* emb, const void* h_local,
+                                int32_t h_local_dtype, int32_t batch, int32_t hidden,
+                                int32_t mlp, const float* w1, const float* b1, const float* w2,
+                                float b2, float theta, float* q_out, int32_t* gate_out,
+                                unsigned long long* full_count,
+                                unsigned long long graph_cond_handle, void* ws, size_t ws_bytes,
+                                void* stream) {
+  return launch_recall(h_prev, emb, h_local, h_local_dtype, batch, hidden, mlp, w1, b1, w2, b2,
+                       theta, q_out, gate_out, full_count, graph_cond_handle, ws, ws_bytes,
+                       stream, 0);
 }

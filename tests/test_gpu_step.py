@@ -30,14 +30,17 @@ def _logical(bits, bt, caps, hkv, d):
     return out
 
 
-def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02):
+def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02, timing=False):
     lay = oda_synth.make_layout(w, extra_tokens=steps + 2, device="cuda", lengths=lengths)
     caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
     rw = oda_synth.make_recall_weights(w, device="cuda", std=recall_std)
     eng = OdaEngine([c[0] for c in caches], [c[1] for c in caches], lay.block_table,
                     w.num_q_heads, (rw.w1, rw.b1, rw.w2, rw.b2), theta, sink=w.sink,
-                    window=w.window, use_conditional=use_conditional)
+                    window=w.window, use_conditional=use_conditional, timing=timing)
     h0 = oda_synth.make_h0(w, device="cuda")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in evs:
+        e.record()
     eng.set_h_prev(h0, 0)
     bt = lay.block_table.cpu().numpy()
     caps = lay.capacity
@@ -52,9 +55,14 @@ def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02):
     for i in range(steps):
         si = oda_synth.make_step_inputs(w, i, device="cuda")
         fill_staging(eng.v, si, [n + i + 1 for n in lengths])
+        if timing:
+            eng.set_events(i, evs)
         eng.launch(i)
         torch.cuda.synchronize()
         assert int(eng.status.item()) == 0
+        if timing:
+            phases = [evs[k].elapsed_time(evs[k + 1]) for k in range(3)]
+            assert all(x >= 0 for x in phases) and phases[0] > 0
         outs = np.stack([eng.layer_out(i, l).cpu().numpy() for l in range(w.layers)])
         q = eng.q_out.cpu().numpy()
         gate = eng.gate.cpu().numpy().astype(bool)
@@ -85,6 +93,12 @@ def test_step_graph_matches_oracle_ragged(use_conditional):
                            prefill=300, steps=6, seed=77, sink=4, window=64)
     n = _run_steps(w, [300, 37, 170], 6, theta=0.0, use_conditional=use_conditional)
     assert 0 < n < 18                      # both paths exercised
+
+
+def test_step_graph_with_timing_events():
+    w = oda_synth.Workload(name="tiny3", layers=2, batch=2, num_q_heads=16, num_kv_heads=8,
+                           prefill=700, steps=4, seed=79, sink=4, window=128)
+    _run_steps(w, [700, 300], 4, theta=0.0, timing=True)
 
 
 def test_step_graph_all_local_and_all_full():
