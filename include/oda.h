@@ -123,6 +123,22 @@ int oda_decode_full(const oda_kv* kv, const void* q, int32_t num_q_heads, float 
                     void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
                     void* stream);
 
+/* Full decode for callers that cannot allocate device memory (no counterpart in the papers;
+ * an engineering addition). Same arguments and results as oda_decode_full, without the
+ * workspace: code running under a CUDA-graph capture mode that forbids allocation calls, or
+ * inside a host framework that owns every device allocation, or that must not risk an
+ * allocation failure mid-step, cannot hand in a cudaMalloc'd buffer. The split partials and
+ * merge tickets then live in a 2 MiB device array inside liboda, held by every GPU that loads
+ * the library until exit; a batch whose workspace (oda_decode_workspace_size) exceeds 2 MiB
+ * returns ODA_ERR_WORKSPACE_TOO_SMALL. The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * Each call clears the array's tickets with an asynchronous memset on `stream` and allocates
+ * nothing. All calls share the one array: calls that overlap on the GPU (different streams,
+ * no ordering between them) race and give wrong results. */
+int oda_decode_full_noalloc(const oda_kv* kv, const void* q, int32_t num_q_heads, float scale,
+                            const int32_t* gate, const void* k_new, const void* v_new,
+                            void* out, int32_t out_dtype, float* lse, void* stream);
+
 /* Keep-block mask ([DA] section 3: the engine rewrites the block table so that only the kept
  * pages reach the attention kernel). keep_blocks: int32 [batch][max_keep] logical page ids,
  * strictly ascending, each <= t / 16; keep_counts: int32 [batch]. Visible positions are the

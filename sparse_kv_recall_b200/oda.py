@@ -87,6 +87,7 @@ _SIGNATURES = {
     "oda_decode_local": (ctypes.c_int, [_KV, _P, _I, _I, _I, _F, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "oda_decode_full": (ctypes.c_int, [_KV, _P, _I, _F, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "oda_decode_blockmask": (ctypes.c_int, [_KV, _P, _I, _F, _P, _P, _I, _P, _I, _P, _P, _SZ, _P]),
+    "oda_decode_full_noalloc": (ctypes.c_int, [_KV, _P, _I, _F, _P, _P, _P, _P, _I, _P, _P]),
     "oda_visible_mask": (ctypes.c_int, [_KV, _I, _I, _I, _P, _P, _P, _I, _P, _I, _P]),
     "oda_recall_score": (ctypes.c_int, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _F, _F, _P, _P, _P,
                                         ctypes.c_ulonglong, _P, _SZ, _P]),
@@ -213,6 +214,17 @@ def oda_decode_full(kv: oda_kv, q, scale: float, out, ws, gate=None, k_new=None,
         _ptr(v_new, torch.bfloat16, "v_new"), _ptr(out, None, "out"), _out_dtype(out),
         _ptr(lse, torch.float32, "lse"), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
         _stream(stream)), "oda_decode_full")
+
+
+def oda_decode_full_noalloc(kv: oda_kv, q, scale: float, out, gate=None, k_new=None, v_new=None,
+                            lse=None, stream=None):
+    """oda_decode_full for callers that cannot allocate: no workspace argument; the library's
+    own per-device scratch array is used (calls that overlap on the GPU race on it)."""
+    _check(load().oda_decode_full_noalloc(
+        ctypes.byref(kv), _ptr(q, torch.bfloat16, "q"), q.shape[1], scale,
+        _ptr(gate, torch.int32, "gate"), _ptr(k_new, torch.bfloat16, "k_new"),
+        _ptr(v_new, torch.bfloat16, "v_new"), _ptr(out, None, "out"), _out_dtype(out),
+        _ptr(lse, torch.float32, "lse"), _stream(stream)), "oda_decode_full_noalloc")
 
 
 def oda_decode_blockmask(kv: oda_kv, q, scale: float, keep_blocks, keep_counts, out, ws,
