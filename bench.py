@@ -57,6 +57,8 @@ def parse_args():
     ap.add_argument("--kernel-reps", type=int, default=28)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-gate-point", action="store_true",
+                    help="skip the 4K-history gate-overhead point")
     ap.add_argument("--quick", action="store_true",
                     help="main timed region only (used for profiler launch lists)")
     ap.add_argument("--no-conditional", action="store_true",
@@ -233,6 +235,101 @@ def launches_per_step(w, phases: int, steps: int, conditional: bool = True) -> i
     return steps * (w.layers + 1) + (phases if conditional else steps) * w.layers
 
 
+def calibrate_theta(s, w, C: int, step: int):
+    """theta = (1 - target rho) quantile of q over C Local-only steps (graphs captured with
+    theta = +inf); returns (theta, next step index)."""
+    qs = []
+    for _ in range(C):
+        s.feed(step)
+        s.eng.launch(step)
+        qs.append(s.eng.q_out.clone())
+        step += 1
+    q = torch.cat(qs).double().cpu().numpy()
+    return float(np.quantile(q, 1.0 - w.target_rho)), step
+
+
+def phase_breakdown(s, w, theta: float, PH: int, step: int, stream):
+    """PH steps of the same graphs with event nodes at the phase boundaries (Local | recall |
+    Full); returns (phase dict, next step index)."""
+    eng = s.eng
+    eng.timing = True
+    eng.set_theta(theta)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(PH)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    gated = []
+    for i in range(PH):
+        before = eng.full_count[1].clone()
+        eng.set_events(step, evs[i])
+        s.feed(step)
+        eng.launch(step)
+        gated.append(before)
+        step += 1
+    torch.cuda.synchronize()
+    counts = torch.stack(gated).cpu().tolist() + [int(eng.full_count[1].item())]
+    ran_full = [counts[i + 1] > counts[i] for i in range(PH)]
+    t_local = [evs[i][0].elapsed_time(evs[i][1]) for i in range(PH)]
+    t_recall = [evs[i][1].elapsed_time(evs[i][2]) for i in range(PH)]
+    t_full = [evs[i][2].elapsed_time(evs[i][3]) for i in range(PH)]
+    t_step = [evs[i][0].elapsed_time(evs[i][3]) for i in range(PH)]
+    full_steps = [i for i in range(PH) if ran_full[i]]
+    local_steps = [i for i in range(PH) if not ran_full[i]]
+    mean = lambda xs: float(np.mean(xs)) if xs else None
+    T_step, T_loc = mean(t_step), mean(t_local)
+    T_full_exec = sum(t_full[i] for i in full_steps) / PH if PH else 0.0
+    gate_over = (T_step - T_loc - T_full_exec) / T_step if T_step else None
+    ctx = np.mean(s.lengths) + step - PH / 2
+    full_launch_bytes = w.batch * (ctx + 1) * w.num_kv_heads * ROW_BYTES
+    local_rows = sum(min(n + step - PH / 2 + 1, w.sink + w.window) for n in s.lengths)
+    eng.timing = False
+    eng.set_theta(theta)
+    return {
+        "steps": PH, "steps_with_full": len(full_steps), "ms_step": T_step, "ms_local_phase": T_loc,
+        "ms_recall": mean(t_recall), "ms_full_phase_when_run": mean([t_full[i] for i in full_steps]),
+        "ms_full_phase_when_skipped": mean([t_full[i] for i in local_steps]),
+        "gate_overhead": gate_over,
+        "gate_overhead_def": "(step - Local phase - executed Full phase) / step; recall and IF "
+                             "node timed without PDL between event nodes",
+        "local_phase_kv_gbs": (w.layers * w.num_kv_heads * local_rows * ROW_BYTES
+                               / (T_loc / 1e3) / 1e9) if T_loc else None,
+        "full_phase_kv_gbs": (w.layers * full_launch_bytes / (mean([t_full[i] for i in full_steps]) / 1e3)
+                              / 1e9) if full_steps else None,
+    }, step
+
+
+def run_gate_point(args, dev, stream, prefill: int = 4096, steps: int = 512):
+    """The gate-overhead point: the default workload's shapes with a short history."""
+    w = oda_synth.scaled(oda_synth.WORKLOADS[args.workload], prefill=prefill,
+                         name=args.workload + "@%d" % prefill)
+    C, W, PH = 256, 8, steps
+    s = Setup(w, 0, C + W + 2 * PH, float("inf"), dev)
+    theta, step = calibrate_theta(s, w, C, 0)
+    s.eng.set_theta(theta)
+    for _ in range(W):
+        s.feed(step)
+        s.eng.launch(step)
+        step += 1
+    fc0 = s.eng.full_count.clone()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(PH):
+        s.feed(step)
+        s.eng.launch(step)
+        step += 1
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    rho = float((s.eng.full_count - fc0)[0].item()) / (w.batch * PH)
+    ph, step = phase_breakdown(s, w, theta, PH, step, stream)
+    assert int(s.eng.status.item()) == 0
+    s.eng.close()
+    return {"workload": w.name, "tokens_per_s": w.batch * PH / (ms / 1e3), "ms_per_step": ms / PH,
+            "rho_realised": rho, "theta": theta, "phases": ph}
+
+
 def run_oda(args, dist: Dist):
     from sparse_kv_recall_b200 import build as B
     from sparse_kv_recall_b200 import oda
@@ -258,14 +355,7 @@ def run_oda(args, dist: Dist):
     # theta for the target Full-call rate: quantile of q over Local-only calibration steps
     theta = w.theta
     if theta is None:
-        qs = []
-        for _ in range(C):
-            s.feed(step)
-            eng.launch(step)
-            qs.append(eng.q_out.clone())
-            step += 1
-        q = torch.cat(qs).double().cpu().numpy()
-        theta = float(np.quantile(q, 1.0 - w.target_rho))
+        theta, step = calibrate_theta(s, w, C, step)
         eng.set_theta(theta)
 
     for _ in range(W):
@@ -326,49 +416,7 @@ def run_oda(args, dist: Dist):
         return result, s
 
     # ---- phase breakdown: same graphs with event nodes at the phase boundaries ----
-    eng.timing = True
-    eng.set_theta(theta)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(PH)]
-    for row in evs:
-        for e in row:
-            e.record(stream)
-    torch.cuda.synchronize()
-    fc0 = eng.full_count.clone()
-    gated = []
-    for i in range(PH):
-        before = eng.full_count[1].clone()
-        eng.set_events(step, evs[i])
-        s.feed(step)
-        eng.launch(step)
-        gated.append(before)
-        step += 1
-    torch.cuda.synchronize()
-    counts = torch.stack(gated).cpu().tolist() + [int(eng.full_count[1].item())]
-    ran_full = [counts[i + 1] > counts[i] for i in range(PH)]
-    t_local = [evs[i][0].elapsed_time(evs[i][1]) for i in range(PH)]
-    t_recall = [evs[i][1].elapsed_time(evs[i][2]) for i in range(PH)]
-    t_full = [evs[i][2].elapsed_time(evs[i][3]) for i in range(PH)]
-    t_step = [evs[i][0].elapsed_time(evs[i][3]) for i in range(PH)]
-    full_steps = [i for i in range(PH) if ran_full[i]]
-    local_steps = [i for i in range(PH) if not ran_full[i]]
-    mean = lambda xs: float(np.mean(xs)) if xs else None
-    T_step, T_loc = mean(t_step), mean(t_local)
-    T_full_exec = sum(t_full[i] for i in full_steps) / PH if PH else 0.0
-    gate_over = (T_step - T_loc - T_full_exec) / T_step if T_step else None
-    ctx = np.mean(s.lengths) + step - PH / 2
-    full_launch_bytes = w.batch * (ctx + 1) * w.num_kv_heads * ROW_BYTES
-    result["phases"] = {
-        "steps": PH, "steps_with_full": len(full_steps), "ms_step": T_step, "ms_local_phase": T_loc,
-        "ms_recall": mean(t_recall), "ms_full_phase_when_run": mean([t_full[i] for i in full_steps]),
-        "ms_full_phase_when_skipped": mean([t_full[i] for i in local_steps]),
-        "gate_overhead": gate_over,
-        "local_phase_kv_gbs": (w.batch * w.layers * w.num_kv_heads * (w.sink + w.window) * ROW_BYTES
-                               / (T_loc / 1e3) / 1e9) if T_loc else None,
-        "full_phase_kv_gbs": (w.layers * full_launch_bytes / (mean([t_full[i] for i in full_steps]) / 1e3)
-                              / 1e9) if full_steps else None,
-    }
-    eng.timing = False
-    eng.set_theta(theta)
+    result["phases"], step = phase_breakdown(s, w, theta, PH, step, stream)
 
     # ---- dominant kernel alone: Full decode at this context, CUDA events per launch ----
     from sparse_kv_recall_b200 import oda as O
@@ -420,6 +468,8 @@ def run_oda(args, dist: Dist):
                          "h2d_bytes_per_step": s.slot,
                          "d2h_bytes_per_step": w.batch * (w.hidden * 4 + 4)}
     assert int(eng.status.item()) == 0, "device status %d" % int(eng.status.item())
+    if not args.no_gate_point and w.name == DEFAULT_WORKLOAD:
+        result["gate_point_4k"] = run_gate_point(args, dev, stream)
     return result, s
 
 

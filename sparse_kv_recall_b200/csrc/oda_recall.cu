@@ -4,11 +4,13 @@
 // same execution stream as Local and the conditional Full pass).
 //
 // q = w2 . GELU(W1^T x + b1) + b2 with x = [h_prev; emb; h_local] (3 * hidden rows of W1).
-// The 3*hidden x mlp weight matrix is split into kRows-row slabs x 64-column tiles, one CTA
-// each, so the whole GPU streams W1 once per call for every sequence of the batch. Per
-// column tile, the last slab CTA to finish (atomic ticket) sums the slabs' partial z in
-// fixed order and applies b1, GELU and w2; the last column tile then forms q, the gate, the
-// counter and the graph condition. Fixed orders make every result bitwise reproducible.
+// The 3*hidden x mlp weight matrix is split into 256-row slabs x 64-column tiles, one CTA
+// each, so the whole GPU streams W1 once per call for every sequence of the batch; each
+// thread holds its 64 W1 values in registers, all loads in flight at once. Per column tile,
+// the last slab CTA to finish (atomic ticket) sums the slabs' partial z in fixed order, one
+// (sequence, column) per thread with 16 loads in flight, and applies b1, GELU and w2; the
+// last column tile then forms q, the gate, the counters and the graph condition. Fixed
+// orders make every result bitwise reproducible.
 #include <math.h>
 
 #include "oda_common.cuh"
@@ -19,9 +21,10 @@ namespace oda {
 constexpr int kRThreads = 256;
 constexpr int kColTile = 64;
 constexpr int kRowGroups = kRThreads / kColTile;  // 4
-constexpr int kRows = 128;                        // rows of W1 per CTA
+constexpr int kRows = 256;                        // rows of W1 per CTA
 constexpr int kRowsPerThread = kRows / kRowGroups;
 constexpr int kBTile = 8;                         // sequences per pass over the slab
+constexpr int kSlabChunk = 16;                    // slab partials in flight per thread
 
 struct RecallWs {
   size_t z_off, q_off, ticket_off, total;
@@ -78,7 +81,7 @@ __device__ __forceinline__ float x_at(const RecallParams& p, int b, int r) {
 __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p) {
   __shared__ float xs[kBTile][kRows];
   __shared__ float red[kRowGroups][kBTile][kColTile];
-  __shared__ float qs[kBTile][2];
+  __shared__ float qs[kRowGroups][2];
   __shared__ int s_last;
   __shared__ unsigned s_any, s_count;
 
@@ -90,17 +93,16 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
   const int nrows = min(kRows, 3 * p.hidden - r0);
   const int gcol = tile * kColTile + col;
 
-  // Slabs that read only h_prev and emb rows may run while the previous kernel (the last
-  // Local layer, which writes h_local) finishes; the others wait for it first.
-  if (r0 + nrows > 2 * p.hidden) griddep_wait();
-  griddep_launch_dependents();
-
   float wv[kRowsPerThread];  // this thread's W1 column over its rows, all loads in flight
 #pragma unroll
   for (int i = 0; i < kRowsPerThread; ++i) {
     const int r = rg + i * kRowGroups;
     wv[i] = r < nrows ? __ldg(&p.w1[(size_t)(r0 + r) * p.mlp + gcol]) : 0.f;
   }
+  // W1 is constant, so its loads above may overlap the previous kernel (the last Local
+  // layer, which writes h_local); slabs that read h_local rows wait for it only now.
+  if (r0 + nrows > 2 * p.hidden) griddep_wait();
+  griddep_launch_dependents();
 
   // ---- partial z of this slab for every sequence ----
   for (int b0 = 0; b0 < p.batch; b0 += kBTile) {
@@ -138,32 +140,32 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int b0 = 0; b0 < p.batch; b0 += kBTile) {
-    const int nb = min(kBTile, p.batch - b0);
-    float zz[kBTile];
+  // Thread (bl, col) sums column gcol of sequence b0 + bl over every slab, kSlabChunk
+  // independent loads in flight at a time, in fixed slab order.
+  const int bl = tid / kColTile;
+  for (int b0 = 0; b0 < p.batch; b0 += kRowGroups) {
+    const int b = b0 + bl;
+    float v = 0.f;
+    if (b < p.batch) {
+      const float* zp = p.z_part + (size_t)b * p.mlp + gcol;
+      const size_t sstride = (size_t)p.batch * p.mlp;
+      float z = 0.f;
+      for (int s0 = 0; s0 < slabs; s0 += kSlabChunk) {
+        float part[kSlabChunk];
 #pragma unroll
-    for (int bb = 0; bb < kBTile; ++bb) zz[bb] = 0.f;
-#pragma unroll 4
-    for (int sl = rg; sl < slabs; sl += kRowGroups) {
+        for (int u = 0; u < kSlabChunk; ++u)
+          part[u] = (s0 + u < slabs) ? __ldcg(zp + (size_t)(s0 + u) * sstride) : 0.f;
 #pragma unroll
-      for (int bb = 0; bb < kBTile; ++bb)
-        if (bb < nb) zz[bb] += __ldcg(&p.z_part[((size_t)sl * p.batch + b0 + bb) * p.mlp + gcol]);
-    }
-#pragma unroll
-    for (int bb = 0; bb < kBTile; ++bb) red[rg][bb][col] = zz[bb];
-    __syncthreads();
-    if (tid < kColTile) {  // warps 0 and 1: one column each
-      for (int bb = 0; bb < nb; ++bb) {
-        const float z = red[0][bb][col] + red[1][bb][col] + red[2][bb][col] + red[3][bb][col] +
-                        p.b1[gcol];
-        float v = gelu_erf(z) * p.w2[gcol];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if ((tid & 31) == 0) qs[bb][tid >> 5] = v;
+        for (int u = 0; u < kSlabChunk; ++u) z += part[u];
       }
+      v = gelu_erf(z + p.b1[gcol]) * p.w2[gcol];
     }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((tid & 31) == 0) qs[bl][(tid >> 5) & 1] = v;
     __syncthreads();
-    if (tid < nb) p.q_part[(size_t)tile * p.batch + b0 + tid] = qs[tid][0] + qs[tid][1];
+    if (tid < kRowGroups && b0 + tid < p.batch)
+      p.q_part[(size_t)tile * p.batch + b0 + tid] = qs[tid][0] + qs[tid][1];
     __syncthreads();
   }
   if (tid == 0) p.tickets[tile] = 0u;
