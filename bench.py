@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gate-point", action="store_true",
                     help="skip the 4K-history gate-overhead point")
+    ap.add_argument("--no-da", action="store_true",
+                    help="skip the block-mask (Declarative Attention) sub-measurement")
     ap.add_argument("--quick", action="store_true",
                     help="main timed region only (used for profiler launch lists)")
     ap.add_argument("--no-conditional", action="store_true",
@@ -299,35 +301,189 @@ def phase_breakdown(s, w, theta: float, PH: int, step: int, stream):
     }, step
 
 
-def run_gate_point(args, dev, stream, prefill: int = 4096, steps: int = 512):
+def timed_steps(s, n: int, step: int, stream):
+    """ms per step over n steps of the engine's current graphs (inputs fed from the pool)."""
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        s.feed(step)
+        s.eng.launch(step)
+        step += 1
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / n, step
+
+
+def gate_cost(s, w, theta: float, n: int, step: int, stream):
+    """Step time of the same PDL-chained graphs (no event nodes inside) at the calibrated
+    theta, at theta = +inf (Local + recall + skipped IF node), at theta = -inf (every step
+    runs Full) and as a Local-only graph; the recall head and the IF machinery cost
+    T(+inf) - T(Local only), the Full phase T(-inf) - T(+inf)."""
+    from sparse_kv_recall_b200 import oda
+    eng = s.eng
+    out = {}
+    fc0 = eng.full_count.clone()
+    for name, th, phases in [("oda", theta, 0), ("theta_plus_inf", math.inf, 0),
+                             ("theta_minus_inf", -math.inf, 0),
+                             ("local_only", math.inf, oda.ODA_PHASE_LOCAL)]:
+        eng.phases = phases
+        eng.set_theta(th)
+        _, step = timed_steps(s, 8, step, stream)            # settle after re-capture
+        if name == "oda":
+            fc0 = eng.full_count.clone()
+        out[name], step = timed_steps(s, n, step, stream)
+        if name == "oda":
+            out["rho_realised"] = float((eng.full_count - fc0)[0].item()) / (w.batch * n)
+    eng.phases = 0
+    eng.set_theta(theta)
+    T = out
+    overhead = T["theta_plus_inf"] - T["local_only"]
+    return {"ms_per_step": {k: v for k, v in T.items() if k.startswith(("oda", "theta", "local"))},
+            "rho_realised": T["rho_realised"],
+            "ms_recall_and_if_node": overhead,
+            "ms_full_phase": T["theta_minus_inf"] - T["theta_plus_inf"],
+            "gate_overhead": overhead / T["oda"],
+            "gate_overhead_def": "(T(theta=+inf) - T(Local-only graph)) / T(calibrated theta): "
+                                 "recall head + IF node per step over the whole step, same "
+                                 "PDL-chained graphs, no event nodes inside"}, step
+
+
+def run_gate_point(args, dev, stream, prefill: int = 4096, steps: int = 256):
     """The gate-overhead point: the default workload's shapes with a short history."""
     w = oda_synth.scaled(oda_synth.WORKLOADS[args.workload], prefill=prefill,
                          name=args.workload + "@%d" % prefill)
-    C, W, PH = 256, 8, steps
-    s = Setup(w, 0, C + W + 2 * PH, float("inf"), dev)
+    C, W = 256, 8
+    s = Setup(w, 0, C + W + 5 * steps + 64, float("inf"), dev)
     theta, step = calibrate_theta(s, w, C, 0)
     s.eng.set_theta(theta)
     for _ in range(W):
         s.feed(step)
         s.eng.launch(step)
         step += 1
-    fc0 = s.eng.full_count.clone()
+    res, step = gate_cost(s, w, theta, steps, step, stream)
+    ph, step = phase_breakdown(s, w, theta, steps, step, stream)
+    assert int(s.eng.status.item()) == 0
+    s.eng.close()
+    res.update({"workload": w.name, "tokens_per_s": w.batch / (res["ms_per_step"]["oda"] / 1e3),
+                "theta": theta, "phases_with_event_nodes": ph})
+    return res
+
+
+def run_da(w, dist: Dist, steps: int, warmup: int, dev: str, stream, e2e: bool = True):
+    """Declarative-Attention block-mask decode: per step and sequence a mode is drawn
+    (global / focus / local), its keep-page list built on the host (da.keep_pages), and the
+    step runs the commit of the step's K/V (oda_kv_append) and the keep-list decode
+    (oda_decode_blockmask). Keep lists, counts, lengths and q/k/v for every step sit in a
+    resident pool (one copy per step); with e2e the same steps run from pinned host memory."""
+    from sparse_kv_recall_b200 import da, oda
+    lengths = oda_synth.prefill_lengths(w)
+    total = warmup + steps + (steps if e2e else 0)
+    lay = oda_synth.make_layout(w, extra_tokens=total + 4, device=dev)
+    kc, vc = oda_synth.make_kv_cache(w, lay, 0, device=dev)
+    maxkeep = lay.block_table.shape[1]
+    B, Hq, Hkv = w.batch, w.num_q_heads, w.num_kv_heads
+    # pool row: seq_lens [B] | counts [B] | keep [B][maxkeep] (int32) | q | k | v (bf16);
+    # the int32 block is padded to 256 bytes so the bf16 tensors start 16-byte aligned
+    n_int = 2 * B + B * maxkeep
+    n_int = (n_int * 4 + 255) // 256 * 256 // 4
+    n_bf = B * Hq * 128 + 2 * B * Hkv * 128
+    row = n_int * 4 + n_bf * 2
+    pool = torch.empty((total, row), dtype=torch.uint8, device=dev)
+    for i in range(total):
+        pos = [n + i for n in lengths]
+        draws = oda_synth.draw_da_modes(w, i, pos)
+        keep, counts = da.keep_lists(draws, pos, maxkeep)
+        ints = np.zeros(n_int, np.int32)
+        ints[:2 * B + B * maxkeep] = np.concatenate([np.array([p + 1 for p in pos], np.int32),
+                                                     counts, keep.reshape(-1)])
+        ints = torch.from_numpy(ints)
+        si = oda_synth.make_step_inputs(w, i, device=dev)
+        pool[i, :n_int * 4].copy_(ints.view(torch.uint8))
+        bf = torch.cat([si.q_local[0].reshape(-1), si.k_local[0].reshape(-1), si.v_local[0].reshape(-1)])
+        pool[i, n_int * 4:].copy_(bf.view(torch.uint8))
+    stage = torch.empty(row, dtype=torch.uint8, device=dev)
+    ints = stage[:n_int * 4].view(torch.int32)
+    seq, counts, keep = ints[:B], ints[B:2 * B], ints[2 * B:2 * B + B * maxkeep].view(B, maxkeep)
+    bfv = stage[n_int * 4:].view(torch.bfloat16)
+    q = bfv[:B * Hq * 128].view(B, Hq, 128)
+    k_new = bfv[B * Hq * 128:B * Hq * 128 + B * Hkv * 128].view(B, Hkv, 128)
+    v_new = bfv[B * Hq * 128 + B * Hkv * 128:].view(B, Hkv, 128)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stats = torch.zeros(2, dtype=torch.int64, device=dev)
+    kv = oda.make_kv(kc, vc, lay.block_table, seq, status, stats)
+    ws = torch.zeros(oda.oda_decode_workspace_size(B, Hkv, Hq), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(128)
+
+    def step(src):
+        stage.copy_(src, non_blocking=True)
+        oda.oda_kv_append(kv, k_new, v_new)
+        oda.oda_decode_blockmask(kv, q, scale, keep, counts, out, ws)
+
+    for i in range(warmup):
+        step(pool[i])
     torch.cuda.synchronize()
+    st0 = stats.clone()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(PH):
-        s.feed(step)
-        s.eng.launch(step)
-        step += 1
+    for i in range(warmup, warmup + steps):
+        step(pool[i])
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
-    rho = float((s.eng.full_count - fc0)[0].item()) / (w.batch * PH)
-    ph, step = phase_breakdown(s, w, theta, PH, step, stream)
-    assert int(s.eng.status.item()) == 0
-    s.eng.close()
-    return {"workload": w.name, "tokens_per_s": w.batch * PH / (ms / 1e3), "ms_per_step": ms / PH,
-            "rho_realised": rho, "theta": theta, "phases": ph}
+    st = (stats - st0).cpu().tolist()
+    res = {"workload": w.name, "steps": steps, "tokens_per_s": B * steps / (ms / 1e3),
+           "ms_per_step": ms / steps, "attended_rows_per_step": st[0] / steps,
+           "kv_gbs": st[0] * ROW_BYTES / (ms / 1e3) / 1e9,
+           "page_gbs": st[1] * PAGE_BYTES / (ms / 1e3) / 1e9,
+           "gpu_launches": 2 * steps}
+    if e2e:
+        host = torch.empty((steps, row), dtype=torch.uint8, pin_memory=True)
+        host.copy_(pool[warmup + steps:])
+        out_h = torch.empty((B, Hq, 128), dtype=torch.float32, pin_memory=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for i in range(steps):
+            step(host[i])
+            out_h.copy_(out, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        res["e2e"] = {"tokens_per_s": B * steps / (a.elapsed_time(b) / 1e3),
+                      "h2d_bytes_per_step": row, "d2h_bytes_per_step": B * Hq * 128 * 4}
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    del kc, vc, pool
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_da_main(args, dist: Dist, w, dev: str):
+    """The block-mask workload as the bench's main line."""
+    stream = torch.cuda.current_stream()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    dist.barrier()
+    r = run_da(oda_synth.scaled(w, seed=w.seed + 1000 * dist.rank), dist, args.steps,
+               max(args.warmup, 3), dev, stream, e2e=not args.no_e2e)
+    dist.barrier()
+    ms = dist.max(r["ms_per_step"] * args.steps)
+    peak, peak_kind = measured_peak()
+    res = {"metric": METRIC, "value": dist.sum(w.batch * args.steps) / (ms / 1e3), "unit": UNIT,
+           "n_gpus": dist.world, "steps": args.steps, "warmup": max(args.warmup, 3),
+           "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+           "config": {"workload": w.name, "layers": 1, "batch_per_gpu": w.batch,
+                      "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads, "prefill": w.prefill,
+                      "modes": "global/focus/local p=%s" % (w.da_probs,), "kv_dtype": "bf16",
+                      "l2": "no flush: ~1.9 GB of kept pages per step >> L2"},
+           "kv_stream": {"gbs": r["kv_gbs"], "frac_of_peak": r["kv_gbs"] / peak, "peak_gbs": peak,
+                         "peak_kind": peak_kind, "attended_rows_per_step": r["attended_rows_per_step"]},
+           "gpu_launches": r["gpu_launches"], "clocks": clocks.stop()}
+    if "e2e" in r:
+        res["e2e"] = {"value": r["e2e"]["tokens_per_s"], "unit": UNIT,
+                      "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
+                      "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"]}
+    return res
 
 
 def run_oda(args, dist: Dist):
@@ -338,14 +494,15 @@ def run_oda(args, dist: Dist):
     dev = "cuda:%d" % dist.local
     torch.cuda.set_device(dist.local)
     w = oda_synth.WORKLOADS[args.workload]
-    if w.mode != "oda":
-        raise SystemExit("bench.py times the ODA step; %s is a block-mask workload" % w.name)
+    if w.mode == "da":
+        return run_da_main(args, dist, w, dev), None
     K, W, C = args.steps, max(args.warmup, 3), args.calib_steps
     if w.theta is not None:
         C = 0
     PH = 0 if args.quick else args.phase_steps
+    GC = 0 if args.quick else 64
     E2E = 0 if (args.quick or args.no_e2e) else min(K, 256)
-    total = C + W + K + PH + E2E
+    total = C + W + K + PH + (4 * GC + 32 if GC else 0) + E2E
     s = Setup(w, dist.rank, total, float("inf") if w.theta is None else w.theta, dev,
               use_conditional=not args.no_conditional)
     eng = s.eng
@@ -417,6 +574,7 @@ def run_oda(args, dist: Dist):
 
     # ---- phase breakdown: same graphs with event nodes at the phase boundaries ----
     result["phases"], step = phase_breakdown(s, w, theta, PH, step, stream)
+    result["gate_cost"], step = gate_cost(s, w, theta, GC, step, stream)
 
     # ---- dominant kernel alone: Full decode at this context, CUDA events per launch ----
     from sparse_kv_recall_b200 import oda as O
@@ -452,6 +610,7 @@ def run_oda(args, dist: Dist):
         gate_h = torch.empty((2, w.batch), dtype=torch.int32, pin_memory=True)
         torch.cuda.synchronize()
         dist.barrier()
+        fc_e = eng.full_count.clone()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for i in range(E2E):
@@ -466,10 +625,16 @@ def run_oda(args, dist: Dist):
         ms_e2e = dist.max(a.elapsed_time(b))
         result["e2e"] = {"value": dist.sum(w.batch * E2E) / (ms_e2e / 1e3), "unit": UNIT,
                          "h2d_bytes_per_step": s.slot,
-                         "d2h_bytes_per_step": w.batch * (w.hidden * 4 + 4)}
+                         "d2h_bytes_per_step": w.batch * (w.hidden * 4 + 4), "steps": E2E,
+                         "rho_realised": float((eng.full_count - fc_e)[0].item()) / (w.batch * E2E),
+                         "note": "its own steps (later in the same decode), so its Full-call "
+                                 "rate differs from the main region's"}
     assert int(eng.status.item()) == 0, "device status %d" % int(eng.status.item())
     if not args.no_gate_point and w.name == DEFAULT_WORKLOAD:
         result["gate_point_4k"] = run_gate_point(args, dev, stream)
+    if not args.no_da and w.name == DEFAULT_WORKLOAD:
+        result["da_blockmask_1m"] = run_da(oda_synth.WORKLOADS["da-1m-b2"], dist, 128, 4, dev,
+                                           stream, e2e=False)
     return result, s
 
 
@@ -622,7 +787,8 @@ def main():
             res = run_reference(args, dist)
         else:
             res, setup = run_oda(args, dist)
-            if dist.rank == 0 and dist.world == 1 and not (args.no_cpu_baseline or args.quick):
+            if (dist.rank == 0 and dist.world == 1 and setup is not None
+                    and not (args.no_cpu_baseline or args.quick)):
                 rho = res["config"]["rho_realised"]
                 del setup
                 torch.cuda.empty_cache()

@@ -58,6 +58,10 @@ const char* oda_status_string(int code);
 /* Library ABI version (major * 100 + minor). */
 int oda_version(void);
 
+/* Text of the most recent CUDA runtime error behind an ODA_ERR_CUDA return on the calling
+ * thread (static storage; "no CUDA error recorded" if none). */
+const char* oda_last_cuda_error(void);
+
 /* ---- the paged KV cache ([ODA] 개발자 관점: the runtime keeps the whole history paged, with a
  *      Local view and a Full view over the same cache) ---------------------------------- */
 typedef struct {
@@ -222,7 +226,11 @@ typedef struct {
   int32_t use_conditional;             /* 1: IF node around the Full phase; 0: Full kernels
                                           always launch and skip ungated sequences on-device */
   int32_t timing_events;               /* 1: event-record nodes at phase boundaries          */
+  int32_t phases;                      /* 0 = whole step; else a mask of ODA_PHASE_* (a step
+                                          without recall or Full is for measurement only)   */
 } oda_step_desc;
+
+enum { ODA_PHASE_LOCAL = 1, ODA_PHASE_RECALL = 2, ODA_PHASE_FULL = 4 };
 
 int oda_step_graph_create(const oda_step_desc* desc, void* stream, oda_step_graph** graph);
 int oda_step_graph_launch(oda_step_graph* graph, void* stream);

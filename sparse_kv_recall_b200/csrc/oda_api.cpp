@@ -1,5 +1,22 @@
 // Status names and version of the liboda C ABI.
+#include <cuda_runtime_api.h>
+
 #include "oda.h"
+
+namespace oda {
+namespace {
+thread_local int g_last_cuda_error = 0;
+}
+void note_cuda_error(int err) {
+  if (err != 0) g_last_cuda_error = err;
+}
+}  // namespace oda
+
+extern "C" const char* oda_last_cuda_error(void) {
+  const int e = oda::g_last_cuda_error;
+  if (e == 0) return "no CUDA error recorded";
+  return cudaGetErrorString(static_cast<cudaError_t>(e));
+}
 
 extern "C" const char* oda_status_string(int code) {
   switch (code) {

@@ -53,5 +53,5 @@ extern "C" int oda_kv_append(const oda_kv* kv, const void* k_new, const void* v_
       kv->block_table, kv->seq_lens, kv->max_blocks_per_seq, kv->num_blocks, kv->num_kv_heads,
       static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), gate,
       kv->dev_status);
-  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
 }

@@ -119,6 +119,15 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ---- host side: CUDA error bookkeeping ---------------------------------------------------
+void note_cuda_error(int err);  // remembered for oda_last_cuda_error()
+
+inline int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return ODA_OK;
+  note_cuda_error(static_cast<int>(e));
+  return ODA_ERR_CUDA;
+}
+
 // ---- host side: per-device launch facts --------------------------------------------------
 struct DeviceInfo {
   int device = -1;

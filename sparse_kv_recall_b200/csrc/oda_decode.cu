@@ -751,7 +751,7 @@ int launch_decode(const oda_kv* kv, int mode, const void* q, int hq, int sink, i
       e = launch_decode_kernel<4>(p, grid, smem, st, pdl != 0);
       break;
   }
-  return e == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 }  // namespace oda
@@ -842,6 +842,6 @@ extern "C" int oda_visible_mask(const oda_kv* kv, int32_t mode, int32_t sink, in
   a.max_keep = max_keep;
   visible_mask_kernel<<<kv->batch, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       a, mask, max_tokens, kv->dev_status);
-  return cudaGetLastError() == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
 }
 

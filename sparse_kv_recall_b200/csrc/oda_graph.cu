@@ -4,9 +4,9 @@
 //
 // Top-level graph:  [ev0] Local+commit x L  [ev1] recall  [ev2] IF(any gate) [ev3]
 // IF body:          Full+gated commit for every layer not marked local-only
-// The recall kernel sets the IF node's condition from the device; the condition resets to
-// 0 at every launch, so a step whose sequences are all Local skips the body entirely, and a
-// step with some gated sequences runs Full kernels that skip the ungated ones on-device.
+// The recall kernel sets the IF node's condition from the device on every step (1 iff any
+// sequence is gated), so a step whose sequences are all Local skips the body entirely, and
+// a step with some gated sequences runs Full kernels that skip the ungated ones on-device.
 #include <stdlib.h>
 
 #include <new>
@@ -52,13 +52,14 @@ int record_event_node(oda_step_graph* g, int i) {
 
 int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditionalHandle cond) {
   const int L = d->num_layers;
+  const int phases = d->phases ? d->phases : (ODA_PHASE_LOCAL | ODA_PHASE_RECALL | ODA_PHASE_FULL);
   int rc;
   if (g->timing && (rc = record_event_node(g, 0)) != ODA_OK) return rc;
   // Programmatic dependent launch between consecutive kernels: each Local layer after the
   // first, the recall head after the last Local layer and each Full layer after the first
   // may start while its predecessor finishes (see the kernels for what they do before
   // waiting). Kernels next to a timing-event node keep ordinary launches.
-  for (int l = 0; l < L; ++l) {
+  for (int l = 0; l < L && (phases & ODA_PHASE_LOCAL); ++l) {
     if (d->sink < 0 || d->window < 1) return ODA_ERR_INVALID_ARG;
     rc = oda::launch_decode(&d->layers[l], ODA_MODE_LOCAL, d->q_local[l], d->num_q_heads,
                             d->sink, d->window, d->scale, nullptr, nullptr, nullptr, 0,
@@ -68,6 +69,12 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
     if (rc != ODA_OK) return rc;
   }
   if (g->timing && (rc = record_event_node(g, 1)) != ODA_OK) return rc;
+  if (!(phases & ODA_PHASE_RECALL)) {
+    if (g->timing)
+      for (int i = 2; i < 4; ++i)
+        if ((rc = record_event_node(g, i)) != ODA_OK) return rc;
+    return ODA_OK;
+  }
   const int hidden = d->num_q_heads * d->layers[0].head_dim;
   rc = oda::launch_recall(d->h_prev, d->emb, d->out[L - 1], ODA_F32, d->layers[0].batch, hidden,
                           d->mlp, d->w1, d->b1, d->w2, d->b2, d->theta, d->q_out, d->gate_out,
@@ -76,6 +83,10 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
   if (rc != ODA_OK) return rc;
   if (g->timing && (rc = record_event_node(g, 2)) != ODA_OK) return rc;
 
+  if (!(phases & ODA_PHASE_FULL)) {
+    if (g->timing && (rc = record_event_node(g, 3)) != ODA_OK) return rc;
+    return ODA_OK;
+  }
   cudaStream_t full_stream = g->cap;
   cudaGraph_t body = nullptr;
   if (d->use_conditional) {
@@ -171,8 +182,9 @@ extern "C" int oda_step_graph_create(const oda_step_desc* desc, void* stream,
         return ODA_ERR_CUDA;
       }
   cudaGraphConditionalHandle cond = 0;
-  if (desc->use_conditional &&
-      cudaGraphConditionalHandleCreate(&cond, g->graph, 0, cudaGraphCondAssignDefault) !=
+  const int phases = desc->phases ? desc->phases : ODA_PHASE_FULL;
+  if (desc->use_conditional && (phases & ODA_PHASE_FULL) &&
+      cudaGraphConditionalHandleCreate(&cond, g->graph, 0, 0) !=
           cudaSuccess) {
     release(g);
     return ODA_ERR_CUDA;
@@ -188,7 +200,7 @@ extern "C" int oda_step_graph_create(const oda_step_desc* desc, void* stream,
   if (rc == ODA_OK && e != cudaSuccess) rc = ODA_ERR_CUDA;
   if (rc == ODA_OK && cudaGraphInstantiate(&g->exec, g->graph, 0) != cudaSuccess) rc = ODA_ERR_CUDA;
   if (rc != ODA_OK) {
-    cudaGetLastError();
+    oda::note_cuda_error(cudaGetLastError());
     release(g);
     return rc;
   }
@@ -198,9 +210,7 @@ extern "C" int oda_step_graph_create(const oda_step_desc* desc, void* stream,
 
 extern "C" int oda_step_graph_launch(oda_step_graph* graph, void* stream) {
   if (graph == nullptr || graph->exec == nullptr) return ODA_ERR_INVALID_ARG;
-  return cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? ODA_OK
-             : ODA_ERR_CUDA;
+  return oda::cuda_status(cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream)));
 }
 
 extern "C" int oda_step_graph_set_events(oda_step_graph* graph, void* ev_start, void* ev_local,

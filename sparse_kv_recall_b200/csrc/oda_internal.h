@@ -8,6 +8,9 @@
 
 namespace oda {
 
+// Remember the most recent CUDA error seen by this thread (reported by oda_last_cuda_error).
+void note_cuda_error(int err);
+
 // Attribute setup for every decode kernel instantiation on the current device; call before
 // stream capture so that nothing but launches is recorded.
 int prepare_decode_kernels();

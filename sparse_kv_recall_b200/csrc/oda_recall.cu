@@ -247,7 +247,7 @@ int launch_recall(const float* h_prev, const float* emb, const void* h_local, in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, recall_kernel, p) == cudaSuccess ? ODA_OK : ODA_ERR_CUDA;
+  return cuda_status(cudaLaunchKernelEx(&cfg, recall_kernel, p));
 }
 
 }  // namespace oda

@@ -73,7 +73,7 @@ class OdaEngine:
                  block_table: torch.Tensor, num_q_heads: int, recall, theta: float, *,
                  sink: int = 4, window: int = 2048, use_conditional: bool = True,
                  timing: bool = False, local_only: Optional[Sequence[int]] = None,
-                 with_lse: bool = False, with_stats: bool = True):
+                 with_lse: bool = False, with_stats: bool = True, phases: int = 0):
         self.L = len(k_caches)
         self.B = block_table.shape[0]
         self.hq = num_q_heads
@@ -84,6 +84,7 @@ class OdaEngine:
         self.k_caches, self.v_caches, self.block_table = list(k_caches), list(v_caches), block_table
         self.w1, self.b1, self.w2, self.b2 = recall
         self.use_conditional, self.timing = use_conditional, timing
+        self.phases = phases
         self.local_only = local_only
         dev = block_table.device
         self.layout = StagingLayout(self.L, self.B, self.hq, self.hkv, self.hidden)
@@ -130,7 +131,8 @@ class OdaEngine:
                 self._layer_out(parity), self.h[parity], v["emb"], self.w1, self.b1, self.w2,
                 self.b2, self.theta, self.q_out, self.gate, self.decode_ws, self.recall_ws,
                 full_count=self.full_count, lse=self.lse, local_only=self.local_only,
-                use_conditional=self.use_conditional, timing_events=self.timing))
+                use_conditional=self.use_conditional, timing_events=self.timing,
+                phases=self.phases))
 
     def set_h_prev(self, h0: torch.Tensor, step: int = 0):
         """h_{t-1} that step `step` will read."""

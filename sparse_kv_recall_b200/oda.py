@@ -32,12 +32,18 @@ ODA_MODE_KEEP = 2
 ODA_STAT_ROWS = 0
 ODA_STAT_PAGES = 1
 ODA_STATS_LEN = 2
+ODA_PHASE_LOCAL = 1
+ODA_PHASE_RECALL = 2
+ODA_PHASE_FULL = 4
 
 
 class OdaError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__("%s failed: %s (%d)" % (where, oda_status_string(code), code))
+        msg = "%s failed: %s (%d)" % (where, oda_status_string(code), code)
+        if code == ODA_ERR_CUDA:
+            msg += ": " + load().oda_last_cuda_error().decode()
+        super().__init__(msg)
 
 
 class oda_kv(ctypes.Structure):
@@ -68,6 +74,7 @@ class oda_step_desc(ctypes.Structure):
         ("decode_ws", ctypes.c_void_p), ("decode_ws_bytes", ctypes.c_size_t),
         ("recall_ws", ctypes.c_void_p), ("recall_ws_bytes", ctypes.c_size_t),
         ("use_conditional", ctypes.c_int32), ("timing_events", ctypes.c_int32),
+        ("phases", ctypes.c_int32),
     ]
 
 
@@ -81,6 +88,7 @@ _SZ = ctypes.c_size_t
 _SIGNATURES = {
     "oda_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "oda_version": (ctypes.c_int, []),
+    "oda_last_cuda_error": (ctypes.c_char_p, []),
     "oda_decode_workspace_size": (ctypes.c_int, [_I, _I, _I, ctypes.POINTER(_SZ)]),
     "oda_recall_workspace_size": (ctypes.c_int, [_I, _I, _I, ctypes.POINTER(_SZ)]),
     "oda_kv_append": (ctypes.c_int, [_KV, _P, _P, _P, _P]),
@@ -275,7 +283,7 @@ class StepGraph:
                  scale: float, q_local, k_local, v_local, q_full, k_full, v_full, out,
                  h_prev, emb, w1, b1, w2, b2: float, theta: float, q_out, gate_out,
                  decode_ws, recall_ws, full_count=None, lse=None, local_only=None,
-                 use_conditional: bool = True, timing_events: bool = False):
+                 use_conditional: bool = True, timing_events: bool = False, phases: int = 0):
         L = len(kvs)
         self._keep = []
         layers = (oda_kv * L)(*kvs)
@@ -305,7 +313,8 @@ class StepGraph:
             decode_ws_bytes=decode_ws.numel() * decode_ws.element_size(),
             recall_ws=_ptr(recall_ws, None, "recall_ws"),
             recall_ws_bytes=recall_ws.numel() * recall_ws.element_size(),
-            use_conditional=int(bool(use_conditional)), timing_events=int(bool(timing_events)))
+            use_conditional=int(bool(use_conditional)), timing_events=int(bool(timing_events)),
+            phases=int(phases))
         self._desc = d
         h = ctypes.c_void_p(0)
         _check(load().oda_step_graph_create(ctypes.byref(d), None, ctypes.byref(h)),

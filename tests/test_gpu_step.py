@@ -113,3 +113,42 @@ def test_pr1_reference_workload_all_steps():
     w = oda_synth.WORKLOADS["pr1-ref-4k"]
     n = _run_steps(w, [w.prefill], w.steps, theta=w.theta)
     assert 0 < n < w.steps
+
+
+def test_local_only_phase_graph():
+    """phases = Local only (a measurement graph): every layer's Local output and commit, no
+    recall head (its outputs stay untouched) and no Full pass."""
+    w = oda_synth.Workload(name="tiny4", layers=2, batch=2, num_q_heads=16, num_kv_heads=8,
+                           prefill=400, steps=2, seed=80, sink=4, window=64)
+    lengths = [400, 150]
+    lay = oda_synth.make_layout(w, extra_tokens=4, device="cuda", lengths=lengths)
+    caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
+    rw = oda_synth.make_recall_weights(w, device="cuda")
+    eng = OdaEngine([c[0] for c in caches], [c[1] for c in caches], lay.block_table,
+                    w.num_q_heads, (rw.w1, rw.b1, rw.w2, rw.b2), -float("inf"), sink=w.sink,
+                    window=w.window, phases=oda.ODA_PHASE_LOCAL)
+    eng.q_out.fill_(7.0)
+    bt = lay.block_table.cpu().numpy()
+    kh = [_logical(oda_synth.bf16_bits(c[0]), bt, lay.capacity, 8, 128) for c in caches]
+    vh = [_logical(oda_synth.bf16_bits(c[1]), bt, lay.capacity, 8, 128) for c in caches]
+    rec = (rw.w1.double().cpu().numpy(), rw.b1.double().cpu().numpy(),
+           rw.w2.double().cpu().numpy(), rw.b2)
+    dec = O.OdaDecoder(kh, vh, lengths, np.zeros((2, w.hidden)), rec, sink=w.sink,
+                       window=w.window, theta=float("inf"))
+    for i in range(2):
+        si = oda_synth.make_step_inputs(w, i, device="cuda")
+        fill_staging(eng.v, si, [n + i + 1 for n in lengths])
+        eng.launch(i)
+        torch.cuda.synchronize()
+        inp = {k: [oda_synth.bf16_bits(x) for x in getattr(si, k)]
+               for k in ("q_local", "k_local", "v_local", "q_full", "k_full", "v_full")}
+        inp["emb"] = si.emb.double().cpu().numpy()
+        ref, _, _, _ = dec.step(inp)
+        outs = np.stack([eng.layer_out(i, l).cpu().numpy() for l in range(w.layers)])
+        assert_attn_close(outs, ref, "local-only step %d" % i)
+    assert torch.all(eng.q_out == 7.0) and eng.full_count.sum().item() == 0
+    for l, (kc, vc) in enumerate(caches):
+        dk = _logical(oda_synth.bf16_bits(kc), bt, lay.capacity, 8, 128)
+        for b, n in enumerate(lengths):
+            assert np.array_equal(dk[b, :, :n + 2], dec.k[l][b, :, :n + 2])
+    eng.close()
