@@ -32,6 +32,7 @@ _P_H0 = 6
 _P_EMB = 7
 _P_LENGTHS = 8
 _P_DAMODE = 9
+_P_GATE_U = 10
 
 
 @dataclasses.dataclass(frozen=True)
@@ -170,6 +171,7 @@ class StepInputs:
     k_full: list
     v_full: list
     emb: torch.Tensor           # fp32 [B][hidden], the current token's embedding
+    gate_u: torch.Tensor = None  # fp32 [B] ~ U[0, 1): draws of the random gate schedule
 
 
 def _bf16_normal(shape, g, device):
@@ -209,7 +211,9 @@ def make_step_inputs(w: Workload, step: int, device="cpu") -> StepInputs:
             cols["v_full"].append(take(nk, (B, Hkv, d)))
     ge = _gen(w.seed, _P_EMB, step, device=device)
     emb = torch.randn((B, w.hidden), generator=ge, device=device, dtype=torch.float32)
-    return StepInputs(emb=emb, **cols)
+    gu = _gen(w.seed, _P_GATE_U, step, device=device)
+    gate_u = torch.rand((B,), generator=gu, device=device, dtype=torch.float32)
+    return StepInputs(emb=emb, gate_u=gate_u, **cols)
 
 
 def make_h0(w: Workload, device="cpu") -> torch.Tensor:

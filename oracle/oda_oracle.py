@@ -95,6 +95,8 @@ def da_mode_positions(mode: int, t: int, focus_offset: int = 0, *, focus_len: in
     if mode == 0:
         regions = [(0, t)]
     elif mode == 1:
+        if focus_offset < 0:
+            raise ValueError("the focused region starts at a position, >= 0")
         regions = [(0, 0), (focus_offset, min(t, focus_offset + focus_len - 1)),
                    (max(0, t - recent + 1), t)]
     elif mode == 2:
@@ -109,6 +111,11 @@ def da_mode_positions(mode: int, t: int, focus_offset: int = 0, *, focus_len: in
         last = min(t, (hi // block) * block + block - 1)
         visible[first:last + 1] = True
     return np.nonzero(visible)[0].astype(np.int64)
+
+
+def shard_positions(t: int, lo: int, hi: int) -> np.ndarray:
+    """One GPU's part of a context-parallel Full: the positions of 0..t inside [lo, hi)."""
+    return np.arange(max(lo, 0), min(hi, t + 1), dtype=np.int64)
 
 
 # ----------------------------------------------------------------------------------------
@@ -158,6 +165,21 @@ def decode_attention(q_heads, k_rows, v_rows, scale: float):
 # ----------------------------------------------------------------------------------------
 # Recall head and gate.
 # ----------------------------------------------------------------------------------------
+def lse_merge(parts):
+    """Combine attention results over disjoint position sets: parts = [(o_r, lse_r)], each o_r
+    normalised over its own set, lse_r its natural-log normaliser (-inf: empty set). The
+    union's result is sum_r e^(lse_r - M) o_r / sum_r e^(lse_r - M), M = max lse_r, with
+    normaliser M + log sum_r e^(lse_r - M); all parts empty gives (0, -inf)."""
+    lses = [float(l) for _, l in parts]
+    m = max(lses)
+    if m == -math.inf:
+        return np.zeros_like(np.asarray(parts[0][0], dtype=np.float64)), -math.inf
+    w = [0.0 if l == -math.inf else math.exp(l - m) for l in lses]
+    total = sum(w)
+    o = sum(wr * np.asarray(o_r, dtype=np.float64) for wr, (o_r, _) in zip(w, parts)) / total
+    return o, m + math.log(total)
+
+
 def gelu(z):
     """Exact GELU: z * Phi(z) = z/2 (1 + erf(z / sqrt 2))."""
     z = np.asarray(z, dtype=np.float64)
@@ -173,6 +195,12 @@ def recall_score(h_prev, emb, h_local, W1, b1, w2, b2):
                         np.asarray(h_local, np.float64)], axis=-1)
     z = x @ np.asarray(W1, np.float64) + np.asarray(b1, np.float64)
     return gelu(z) @ np.asarray(w2, np.float64) + float(b2)
+
+
+def random_schedule_gate(u, rho: float):
+    """[ODA] 주요 결과, the random-timing ablation: Full is called with probability rho at
+    each (sequence, step), independently of the state; u are the caller's uniform draws."""
+    return np.asarray(u, dtype=np.float64) < rho
 
 
 def gate(q, theta: float = DEFAULT_THETA):
@@ -208,7 +236,9 @@ def attention_cost_ratio(n: int, out_len: int, rho: float, sink: int = DEFAULT_S
 class OdaDecoder:
     """The ODA step ([ODA] 접근 방법 and 개발자 관점), over an attention-only stack whose
     per-layer Q/K/V are given as inputs:
-      1. Local at every layer, over the prior cache plus the Local K/V at slot t;
+      1. Local at every layer, over the prior cache plus the Local K/V at slot t (a layer
+         outside the Local restriction -- hybrid backbones restrict only some layers, [ODA]
+         개발자 관점 -- attends all of 0..t here too; s and w may differ per layer);
       2. q_t from the recall head on (h_{t-1}, E(x_t), last layer's Local output);
       3. where q_t > theta, Full at every layer over the same prior cache plus the Full
          K/V at slot t, replacing the Local result;
@@ -216,13 +246,19 @@ class OdaDecoder:
     The cache is kept in logical position order, bf16 bits: k[l][b][g][p][:]."""
 
     def __init__(self, k_hist_bits, v_hist_bits, lengths, h_prev, recall, *,
-                 sink=DEFAULT_SINK, window=DEFAULT_WINDOW, theta=DEFAULT_THETA, scale=None):
+                 sink=DEFAULT_SINK, window=DEFAULT_WINDOW, theta=DEFAULT_THETA, scale=None,
+                 local_layers=None, sinks=None, windows=None, random_rho=None):
         self.k = [np.array(x, dtype=np.uint16) for x in k_hist_bits]   # per layer [B][Hkv][cap][d]
         self.v = [np.array(x, dtype=np.uint16) for x in v_hist_bits]
         self.lengths = list(lengths)
         self.h_prev = np.asarray(h_prev, dtype=np.float64)
         self.W1, self.b1, self.w2, self.b2 = recall
         self.sink, self.window, self.theta = sink, window, theta
+        L = len(self.k)
+        self.local_layers = [True] * L if local_layers is None else [bool(x) for x in local_layers]
+        self.sinks = [sink] * L if sinks is None else list(sinks)
+        self.windows = [window] * L if windows is None else list(windows)
+        self.random_rho = random_rho     # not None: the random-timing ablation decides
         d = self.k[0].shape[-1]
         self.scale = 1.0 / math.sqrt(d) if scale is None else scale
 
@@ -242,7 +278,8 @@ class OdaDecoder:
 
     def step(self, inp, gate_hint=None, near=1e-3):
         """inp: dict of bf16-bit arrays q_local/k_local/v_local/q_full/k_full/v_full, each a
-        list over layers of [B][H][d], and emb fp64 [B][D]. gate_hint: the device's gate, used
+        list over layers of [B][H][d], emb fp64 [B][D] and, for the random schedule, gate_u
+        [B]. gate_hint: the device's gate, used
         only where |q - theta| < near so that a rounding-level tie cannot fork the history.
         Returns (out [L][B][Hq][d], lse [L][B][Hq], q [B], gate [B])."""
         L = len(self.k)
@@ -254,14 +291,19 @@ class OdaDecoder:
         for layer in range(L):
             for b in range(B):
                 t = self.lengths[b]
-                pos = local_positions(t, self.sink, self.window)
+                if self.local_layers[layer]:
+                    pos = local_positions(t, self.sinks[layer], self.windows[layer])
+                else:
+                    pos = full_positions(t)
                 out[layer, b], lse[layer, b] = self._attend(
                     layer, b, t, pos, inp["q_local"][layer][b],
                     inp["k_local"][layer][b], inp["v_local"][layer][b])
         h_local = out[L - 1].reshape(B, Hq * d)
         q = recall_score(self.h_prev, inp["emb"], h_local, self.W1, self.b1, self.w2, self.b2)
         g = gate(q, self.theta)
-        if gate_hint is not None:
+        if self.random_rho is not None:
+            g = random_schedule_gate(inp["gate_u"], self.random_rho)
+        elif gate_hint is not None:
             hint = np.asarray(gate_hint, dtype=bool)
             tie = np.abs(q - self.theta) < near
             g = np.where(tie, hint, g)

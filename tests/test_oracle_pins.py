@@ -80,6 +80,11 @@ def test_keep_list_validation(bad):
         O.keep_positions(100, bad)   # page 7 starts at 112 > t = 100
 
 
+def test_da_focus_offset_must_be_a_position():
+    with pytest.raises(ValueError):
+        O.da_mode_positions(1, 100, -1)
+
+
 def test_da_modes_closed_forms():
     t = 100_000
     assert np.array_equal(O.da_mode_positions(0, t), O.full_positions(t))
@@ -179,13 +184,39 @@ def test_split_then_lse_merge_equals_whole():
     d = 64
     q, K, V = r.standard_normal(d), r.standard_normal((300, d)), r.standard_normal((300, d))
     o, l = O.softmax_attention(q, K, V, 0.125)
-    cuts = [0, 7, 120, 121, 300]
+    cuts = [0, 7, 120, 121, 121, 300]                   # one empty part in the middle
     parts = [O.softmax_attention(q, K[a:b], V[a:b], 0.125) for a, b in zip(cuts, cuts[1:])]
     m = max(p[1] for p in parts)
     wts = np.array([math.exp(p[1] - m) for p in parts])
     merged = sum(w * p[0] for w, p in zip(wts, parts)) / wts.sum()
     np.testing.assert_allclose(merged, o, atol=1e-12)
     assert abs(m + math.log(wts.sum()) - l) < 1e-12
+    # the oracle's merge is the same identity: unsplit attention, whatever the cut order
+    for perm in ([0, 1, 2, 3, 4], [4, 2, 0, 3, 1]):
+        om, lm = O.lse_merge([parts[i] for i in perm])
+        np.testing.assert_allclose(om, o, atol=1e-12)
+        assert abs(lm - l) < 1e-12
+    oe, le = O.lse_merge([(np.zeros(d), -math.inf), (np.zeros(d), -math.inf)])
+    assert np.array_equal(oe, np.zeros(d)) and le == -math.inf
+
+
+def test_shards_tile_the_history():
+    for t in (0, 15, 16, 1000):
+        cuts = [0, 16, 48, 512, 1 << 30]
+        got = np.concatenate([O.shard_positions(t, a, b) for a, b in zip(cuts, cuts[1:])])
+        assert np.array_equal(got, np.arange(t + 1))        # disjoint, complete, in order
+    assert O.shard_positions(10, 16, 32).size == 0          # a shard past t is empty
+
+
+def test_random_schedule_gate_counts():
+    u = _rng(8).random(10_000)
+    assert not O.random_schedule_gate(u, 0.0).any()
+    assert O.random_schedule_gate(u, 1.0).all()             # u in [0, 1)
+    us = np.sort(u)
+    for rho in (0.125, 0.416, 0.5):
+        g = O.random_schedule_gate(u, rho)
+        assert g.sum() == np.searchsorted(us, rho)          # brute count of draws below rho
+        assert np.all(O.random_schedule_gate(u, rho + 0.1) >= g)   # monotone in rho
 
 
 # ---------------------------------------------------------------- recall head and gate
@@ -289,7 +320,7 @@ def _tiny(layers=2, batch=2, Hq=4, Hkv=2, d=16, n=40, s=2, w=8):
     return wl
 
 
-def _decoder(wl, theta):
+def _decoder(wl, theta, **kw):
     lay = oda_synth.make_layout(wl, extra_tokens=8)
     ks, vs = [], []
     for layer in range(wl.layers):
@@ -309,7 +340,7 @@ def _decoder(wl, theta):
     rw = oda_synth.make_recall_weights(wl, std=0.3)
     rec = (rw.w1.double().numpy(), rw.b1.double().numpy(), rw.w2.double().numpy(), rw.b2)
     dec = O.OdaDecoder(ks, vs, oda_synth.prefill_lengths(wl), oda_synth.make_h0(wl).double().numpy(),
-                       rec, sink=wl.sink, window=wl.window, theta=theta)
+                       rec, sink=wl.sink, window=wl.window, theta=theta, **kw)
     return dec, ks, vs, rw
 
 
@@ -394,3 +425,50 @@ def test_gate_hint_only_breaks_near_ties():
     _, _, q2, g2 = dec.step(inp, gate_hint=[True, not (q[1] > theta)])
     assert g2[0]                              # tie: the hint decides
     assert g2[1] == (q[1] > theta) or abs(q[1] - theta) < 1e-3
+
+
+@pytest.mark.parametrize("theta,path", [(math.inf, "local"), (-math.inf, "full")])
+def test_step_per_layer_access_range(theta, path):
+    """Hybrid backbones restrict only some layers to Local ([ODA] 개발자 관점): layer 1 is
+    unrestricted (attends 0..t in the Local attempt too); layers 0 and 2 have their own s and
+    w. Each layer is checked against SDPA with the mask built by slicing, and the recompute
+    attends everything at every layer."""
+    wl = _tiny(layers=3, n=40, s=2, w=8)
+    sinks, windows = [2, 5, 0], [8, 8, 3]
+    dec, ks, vs, _ = _decoder(wl, theta, local_layers=[1, 0, 1], sinks=sinks, windows=windows)
+    for step in range(2):
+        inp = _inp(wl, step)
+        lens = list(dec.lengths)
+        out, _, _, g = dec.step(inp)
+        assert np.all(g == (path == "full"))
+        for layer in range(wl.layers):
+            for b in range(wl.batch):
+                t = lens[b]
+                if path == "full" or layer == 1:
+                    pos = np.arange(t + 1)
+                else:
+                    pos = _local_by_slicing(t, sinks[layer], windows[layer])
+                ref = _sdpa_step(ks[layer][b], vs[layer][b], t, inp["q_" + path][layer][b],
+                                 inp["k_" + path][layer][b], inp["v_" + path][layer][b], pos,
+                                 wl.head_dim)
+                np.testing.assert_allclose(out[layer, b], ref, atol=1e-12)
+                assert np.array_equal(dec.k[layer][b, :, t], inp["k_" + path][layer][b])
+                ks[layer][b, :, t] = inp["k_" + path][layer][b]
+                vs[layer][b, :, t] = inp["v_" + path][layer][b]
+
+
+def test_window_of_one_sees_only_the_new_token():
+    """s = 0, w = 1: the only visible row is the one just written, so o = v_new exactly."""
+    wl = _tiny(layers=2, n=37)
+    dec, _, _, _ = _decoder(wl, math.inf, sinks=[0, 0], windows=[1, 1])
+    inp = _inp(wl, 0)
+    out, lse, _, _ = dec.step(inp)
+    G = wl.num_q_heads // wl.num_kv_heads
+    for layer in range(2):
+        for b in range(wl.batch):
+            for h in range(wl.num_q_heads):
+                v = O.widen_bf16(inp["v_local"][layer][b][h // G])
+                assert np.array_equal(out[layer, b, h], v)
+                s = float(O.widen_bf16(inp["q_local"][layer][b][h]) @
+                          O.widen_bf16(inp["k_local"][layer][b][h // G])) / math.sqrt(wl.head_dim)
+                assert lse[layer, b, h] == pytest.approx(s, abs=1e-12)
