@@ -349,6 +349,82 @@ def gate_cost(s, w, theta: float, n: int, step: int, stream):
                                  "PDL-chained graphs, no event nodes inside"}, step
 
 
+def step_variants(s, w, theta: float, rho: float, n: int, step: int, stream):
+    """Two variants of the same step graphs, timed like the main region:
+    * the random-timing ablation at the realised Full-call rate rho (gate = u < rho on the
+      step's uniform draws, no recall head);
+    * a hybrid access range: every 4th layer outside the Local restriction (it attends its
+      whole history in the Local pass too), the rest Local-first as usual."""
+    eng = s.eng
+    res = {}
+    for name, kw in [("random_schedule_matched_rho", {"random_rho": rho}),
+                     ("hybrid_every_4th_layer_full", {"local_layers": [0 if l % 4 == 3 else 1
+                                                                       for l in range(w.layers)]})]:
+        eng.random_rho = kw.get("random_rho")
+        eng.local_layers = kw.get("local_layers")
+        eng.set_theta(theta)
+        _, step = timed_steps(s, 8, step, stream)
+        fc0 = eng.full_count.clone()
+        ms, step = timed_steps(s, n, step, stream)
+        res[name] = {"steps": n, "ms_per_step": ms, "tokens_per_s": w.batch / (ms / 1e3),
+                     "rho_realised": float((eng.full_count - fc0)[0].item()) / (w.batch * n)}
+    res["hybrid_every_4th_layer_full"]["layers_outside_restriction"] = w.layers // 4
+    eng.random_rho, eng.local_layers = None, None
+    eng.set_theta(theta)
+    return res, step
+
+
+def cp_emulation(s, w, stream, reps: int = 10):
+    """Context-parallel Full on one GPU: the history split into R page-aligned shards
+    (cp.shard_bounds), each shard's SHARD decode timed alone -- the Full work one GPU of an
+    R-GPU group would do -- plus the LSE merge of R partials. The all-gather between GPUs is
+    not part of it (one GPU here)."""
+    from sparse_kv_recall_b200 import cp, oda
+    eng = s.eng
+    kv, q = eng.kvs[min(1, w.layers - 1)], eng.v["q_full_%d" % min(1, w.layers - 1)]
+    B, Hq = w.batch, w.num_q_heads
+    dev = q.device
+    cap = int(eng.seq_lens.max().item())
+
+    def time_it(fn):
+        # reps launches captured in one CUDA graph, so that host launch cost (ctypes and the
+        # launch call, ~10 us) cannot hide a short kernel's device time
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / reps
+
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device=dev)
+    full_ms = time_it(lambda: oda.oda_decode_full(kv, q, eng.scale, out, eng.decode_ws))
+    res = {"context_tokens": cap, "full_ms": full_ms, "note": "per-GPU shard decode and merge "
+           "timed on one GPU (%d launches per CUDA graph, no PDL); the NCCL all-gather (%d B "
+           "per sequence per rank) is not timed" % (reps, Hq * 129 * 4)}
+    for R in (2, 4, 8):
+        o_all = torch.empty(R, B, Hq, 128, dtype=torch.float32, device=dev)
+        l_all = torch.empty(R, B, Hq, dtype=torch.float32, device=dev)
+        shard_ms = []
+        for r, (lo, hi) in enumerate(cp.shard_bounds(cap, R)):
+            vis = oda.shard_visibility(lo, hi)
+            shard_ms.append(time_it(lambda: oda.oda_decode(kv, vis, q, eng.scale, o_all[r],
+                                                           eng.decode_ws, lse=l_all[r])))
+        merge_ms = time_it(lambda: oda.oda_merge_partials(o_all, l_all, out))
+        res["cp%d" % R] = {"shard_ms_max": max(shard_ms), "shard_ms_min": min(shard_ms),
+                           "merge_ms": merge_ms,
+                           "full_speedup_excl_allgather": full_ms / (max(shard_ms) + merge_ms)}
+    return res
+
+
 def run_gate_point(args, dev, stream, prefill: int = 4096, steps: int = 256):
     """The gate-overhead point: the default workload's shapes with a short history."""
     w = oda_synth.scaled(oda_synth.WORKLOADS[args.workload], prefill=prefill,
@@ -370,12 +446,15 @@ def run_gate_point(args, dev, stream, prefill: int = 4096, steps: int = 256):
     return res
 
 
-def run_da(w, dist: Dist, steps: int, warmup: int, dev: str, stream, e2e: bool = True):
+def run_da(w, dist: Dist, steps: int, warmup: int, dev: str, stream, e2e: bool = True,
+           device_modes: bool = False):
     """Declarative-Attention block-mask decode: per step and sequence a mode is drawn
     (global / focus / local), its keep-page list built on the host (da.keep_pages), and the
     step runs the commit of the step's K/V (oda_kv_append) and the keep-list decode
     (oda_decode_blockmask). Keep lists, counts, lengths and q/k/v for every step sit in a
-    resident pool (one copy per step); with e2e the same steps run from pinned host memory."""
+    resident pool (one copy per step); with e2e the same steps run from pinned host memory.
+    device_modes: the step carries only each sequence's declared mode and focus offset, and
+    oda_decode compiles them into page runs on the device (no keep list exists)."""
     from sparse_kv_recall_b200 import da, oda
     lengths = oda_synth.prefill_lengths(w)
     total = warmup + steps + (steps if e2e else 0)
@@ -383,9 +462,11 @@ def run_da(w, dist: Dist, steps: int, warmup: int, dev: str, stream, e2e: bool =
     kc, vc = oda_synth.make_kv_cache(w, lay, 0, device=dev)
     maxkeep = lay.block_table.shape[1]
     B, Hq, Hkv = w.batch, w.num_q_heads, w.num_kv_heads
-    # pool row: seq_lens [B] | counts [B] | keep [B][maxkeep] (int32) | q | k | v (bf16);
-    # the int32 block is padded to 256 bytes so the bf16 tensors start 16-byte aligned
-    n_int = 2 * B + B * maxkeep
+    # pool row: seq_lens [B] | counts [B] | keep [B][maxkeep] (int32) | q | k | v (bf16), or
+    # with device_modes seq_lens [B] | modes [B] | offsets [B]; the int32 block is padded to
+    # 256 bytes so the bf16 tensors start 16-byte aligned
+    n_used = 3 * B if device_modes else 2 * B + B * maxkeep
+    n_int = n_used
     n_int = (n_int * 4 + 255) // 256 * 256 // 4
     n_bf = B * Hq * 128 + 2 * B * Hkv * 128
     row = n_int * 4 + n_bf * 2
@@ -393,10 +474,14 @@ def run_da(w, dist: Dist, steps: int, warmup: int, dev: str, stream, e2e: bool =
     for i in range(total):
         pos = [n + i for n in lengths]
         draws = oda_synth.draw_da_modes(w, i, pos)
-        keep, counts = da.keep_lists(draws, pos, maxkeep)
         ints = np.zeros(n_int, np.int32)
-        ints[:2 * B + B * maxkeep] = np.concatenate([np.array([p + 1 for p in pos], np.int32),
-                                                     counts, keep.reshape(-1)])
+        lens = np.array([p + 1 for p in pos], np.int32)
+        if device_modes:
+            ints[:n_used] = np.concatenate([lens, [d.mode for d in draws],
+                                            [d.focus_offset for d in draws]])
+        else:
+            keep, counts = da.keep_lists(draws, pos, maxkeep)
+            ints[:n_used] = np.concatenate([lens, counts, keep.reshape(-1)])
         ints = torch.from_numpy(ints)
         si = oda_synth.make_step_inputs(w, i, device=dev)
         pool[i, :n_int * 4].copy_(ints.view(torch.uint8))
@@ -404,7 +489,12 @@ def run_da(w, dist: Dist, steps: int, warmup: int, dev: str, stream, e2e: bool =
         pool[i, n_int * 4:].copy_(bf.view(torch.uint8))
     stage = torch.empty(row, dtype=torch.uint8, device=dev)
     ints = stage[:n_int * 4].view(torch.int32)
-    seq, counts, keep = ints[:B], ints[B:2 * B], ints[2 * B:2 * B + B * maxkeep].view(B, maxkeep)
+    seq = ints[:B]
+    if device_modes:
+        vis = oda.da_visibility(ints[B:2 * B], ints[2 * B:3 * B], focus_len=w.da_focus_len,
+                                recent=w.da_recent, local_len=w.da_local_len)
+    else:
+        counts, keep = ints[B:2 * B], ints[2 * B:2 * B + B * maxkeep].view(B, maxkeep)
     bfv = stage[n_int * 4:].view(torch.bfloat16)
     q = bfv[:B * Hq * 128].view(B, Hq, 128)
     k_new = bfv[B * Hq * 128:B * Hq * 128 + B * Hkv * 128].view(B, Hkv, 128)
@@ -419,7 +509,10 @@ def run_da(w, dist: Dist, steps: int, warmup: int, dev: str, stream, e2e: bool =
     def step(src):
         stage.copy_(src, non_blocking=True)
         oda.oda_kv_append(kv, k_new, v_new)
-        oda.oda_decode_blockmask(kv, q, scale, keep, counts, out, ws)
+        if device_modes:
+            oda.oda_decode(kv, vis, q, scale, out, ws)
+        else:
+            oda.oda_decode_blockmask(kv, q, scale, keep, counts, out, ws)
 
     for i in range(warmup):
         step(pool[i])
@@ -433,7 +526,9 @@ def run_da(w, dist: Dist, steps: int, warmup: int, dev: str, stream, e2e: bool =
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     st = (stats - st0).cpu().tolist()
-    res = {"workload": w.name, "steps": steps, "tokens_per_s": B * steps / (ms / 1e3),
+    res = {"workload": w.name, "keep_spec": "device-compiled modes (%d B per step)" % (3 * 4 * B)
+           if device_modes else "host keep lists (%d B per step)" % (4 * (2 * B + B * maxkeep)),
+           "steps": steps, "tokens_per_s": B * steps / (ms / 1e3),
            "ms_per_step": ms / steps, "attended_rows_per_step": st[0] / steps,
            "kv_gbs": st[0] * ROW_BYTES / (ms / 1e3) / 1e9,
            "page_gbs": st[1] * PAGE_BYTES / (ms / 1e3) / 1e9,
@@ -502,7 +597,8 @@ def run_oda(args, dist: Dist):
     PH = 0 if args.quick else args.phase_steps
     GC = 0 if args.quick else 64
     E2E = 0 if (args.quick or args.no_e2e) else min(K, 256)
-    total = C + W + K + PH + (4 * GC + 32 if GC else 0) + E2E
+    VAR = 0 if args.quick else 128
+    total = C + W + K + PH + (4 * GC + 32 if GC else 0) + E2E + (2 * VAR + 16 if VAR else 0)
     s = Setup(w, dist.rank, total, float("inf") if w.theta is None else w.theta, dev,
               use_conditional=not args.no_conditional)
     eng = s.eng
@@ -575,6 +671,7 @@ def run_oda(args, dist: Dist):
     # ---- phase breakdown: same graphs with event nodes at the phase boundaries ----
     result["phases"], step = phase_breakdown(s, w, theta, PH, step, stream)
     result["gate_cost"], step = gate_cost(s, w, theta, GC, step, stream)
+    result["variants"], step = step_variants(s, w, theta, rho, VAR, step, stream)
 
     # ---- dominant kernel alone: Full decode at this context, CUDA events per launch ----
     from sparse_kv_recall_b200 import oda as O
@@ -601,6 +698,9 @@ def run_oda(args, dist: Dist):
                           "frac": achieved / peak, "traffic": traffic,
                           "algorithmic_bytes": alg, "ms_per_launch": dur,
                           "peak_kind": peak_kind + " (burst copy; kernel timed alone)"}
+
+    if w.name == DEFAULT_WORKLOAD:
+        result["context_parallel_1gpu"] = cp_emulation(s, w, stream)
 
     # ---- end to end through the same API: host inputs in, selected output out ----
     if E2E:
@@ -635,6 +735,8 @@ def run_oda(args, dist: Dist):
     if not args.no_da and w.name == DEFAULT_WORKLOAD:
         result["da_blockmask_1m"] = run_da(oda_synth.WORKLOADS["da-1m-b2"], dist, 128, 4, dev,
                                            stream, e2e=False)
+        result["da_device_modes_1m"] = run_da(oda_synth.WORKLOADS["da-1m-b2"], dist, 128, 4, dev,
+                                              stream, e2e=False, device_modes=True)
     return result, s
 
 

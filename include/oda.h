@@ -45,11 +45,16 @@ enum {
                                      treated as empty                                      */
   ODA_DEV_BAD_KEEP_LIST = 3,      /* keep entry not strictly ascending or after page t/16,
                                      or keep_counts[b] outside [0, max_keep]: entry skipped */
-  ODA_DEV_TIMEOUT = 4             /* a bounded device wait gave up                          */
+  ODA_DEV_TIMEOUT = 4,            /* a bounded device wait gave up                          */
+  ODA_DEV_BAD_DA = 5              /* DA mode not ODA_DA_*, or a negative focus offset:
+                                     sequence treated as empty                              */
 };
 
 enum { ODA_F32 = 0, ODA_BF16 = 1 };                               /* output / input dtypes */
-enum { ODA_MODE_LOCAL = 0, ODA_MODE_FULL = 1, ODA_MODE_KEEP = 2 }; /* visible-set rules    */
+enum {                                                            /* visible-set rules    */
+  ODA_MODE_LOCAL = 0, ODA_MODE_FULL = 1, ODA_MODE_KEEP = 2, ODA_MODE_DA = 3, ODA_MODE_SHARD = 4
+};
+enum { ODA_DA_GLOBAL = 0, ODA_DA_FOCUS = 1, ODA_DA_LOCAL = 2 };   /* [DA] declared modes   */
 enum { ODA_STAT_ROWS = 0, ODA_STAT_PAGES = 1, ODA_STATS_LEN = 2 };
 
 /* Returns a static, human-readable name for any status code above. */
@@ -162,6 +167,69 @@ int oda_visible_mask(const oda_kv* kv, int32_t mode, int32_t sink, int32_t windo
                      const int32_t* keep_counts, int32_t max_keep, uint8_t* mask,
                      int32_t max_tokens, void* stream);
 
+/* ---- one entry point for every visibility rule ---------------------------------------
+ * oda_visibility selects the visible set; fields a mode does not use are ignored.
+ *   LOCAL : sink >= 0, window >= 1 (as oda_decode_local)
+ *   FULL  : gate nullable (as oda_decode_full)
+ *   KEEP  : keep_blocks / keep_counts / max_keep (as oda_decode_blockmask)
+ *   DA    : [DA] section 3 -- each sequence declares one mode, compiled on the device into
+ *           ascending runs of kept pages (no keep list is built or uploaded):
+ *             ODA_DA_GLOBAL every page 0..t/16;
+ *             ODA_DA_FOCUS  page 0, the pages of [da_focus_offsets[b], + da_focus_len) and
+ *                           the pages of the da_recent latest positions;
+ *             ODA_DA_LOCAL  the pages of the da_local_len latest positions;
+ *           every position of a kept page up to t is visible. da_modes / da_focus_offsets:
+ *           device int32 [batch]; sizes in tokens, >= 1. A mode outside ODA_DA_* or a
+ *           negative focus offset makes the sequence empty and sets ODA_DEV_BAD_DA.
+ *   SHARD : positions [pos_lo, pos_hi) of 0..t (pos_lo, pos_hi multiples of 16, pos_lo >= 0,
+ *           pos_hi > pos_lo): one GPU's share of a context-parallel Full; gate nullable. A
+ *           sequence with nothing in the range gets out = 0, lse = -inf, which
+ *           oda_merge_partials treats as an empty part. */
+typedef struct {
+  int32_t mode;                       /* ODA_MODE_*                                         */
+  int32_t sink, window;               /* LOCAL                                              */
+  const int32_t* gate;                /* FULL, SHARD: nullable int32 [batch]                */
+  const int32_t* keep_blocks;         /* KEEP                                               */
+  const int32_t* keep_counts;
+  int32_t max_keep;
+  const int32_t* da_modes;            /* DA                                                 */
+  const int32_t* da_focus_offsets;
+  int32_t da_focus_len, da_recent, da_local_len;
+  int32_t pos_lo, pos_hi;             /* SHARD                                              */
+} oda_visibility;
+
+/* Decode attention under any rule (arguments and results as oda_decode_local). k_new /
+ * v_new (nullable) commit slot t and attend it there; they are rejected for KEEP and DA,
+ * whose kept set need not hold slot t, and in SHARD mode only the GPU whose range holds t
+ * writes the slot. */
+int oda_decode(const oda_kv* kv, const oda_visibility* vis, const void* q, int32_t num_q_heads,
+               float scale, const void* k_new, const void* v_new, void* out, int32_t out_dtype,
+               float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Plan export under any rule (as oda_visible_mask). */
+int oda_visible_mask_ex(const oda_kv* kv, const oda_visibility* vis, uint8_t* mask,
+                        int32_t max_tokens, void* stream);
+
+/* LSE merge of the partial results of one decode split over num_parts disjoint position
+ * ranges (context-parallel Full: one part per GPU, gathered into one buffer):
+ *   o_parts   : fp32 [num_parts][batch][num_q_heads][128], each normalised over its range
+ *   lse_parts : fp32 [num_parts][batch][num_q_heads], natural log; -inf marks an empty part
+ * out[b][h] = sum_r e^(lse_r - M) o_r / sum_r e^(lse_r - M) with M = max_r lse_r, and
+ * lse[b][h] (nullable) = M + log sum_r e^(lse_r - M); all parts empty gives 0 and -inf.
+ * Parts are summed in index order (deterministic). With a non-null gate (int32 [batch]),
+ * sequences with gate[b] == 0 keep their out / lse rows. out_dtype: ODA_F32 or ODA_BF16. */
+int oda_merge_partials(const float* o_parts, const float* lse_parts, int32_t num_parts,
+                       int32_t batch, int32_t num_q_heads, const int32_t* gate, void* out,
+                       int32_t out_dtype, float* lse, void* stream);
+
+/* Random gate schedule ([ODA] 주요 결과: the ablation that calls Full at the same realised
+ * rate as ODA but at random steps): gate_out[b] = 1 iff u[b] < rho, for caller-drawn uniform
+ * variates u (device fp32 [batch], in [0, 1)). full_count and graph_cond_handle behave as in
+ * oda_recall_score. rho in [0, 1]. */
+int oda_gate_schedule(const float* u, int32_t batch, float rho, int32_t* gate_out,
+                      unsigned long long* full_count, unsigned long long graph_cond_handle,
+                      void* stream);
+
 /* ---- K4: recall head and gate ([ODA] 접근 방법: q_t = R(h_{t-1}, E(x_t), h^L_t); Full iff
  *      q_t > theta; 개발자 관점: evaluated in FP32 on the GPU, no routing sync) ----------
  *   h_prev  : fp32 [batch][hidden]  previous step's selected last-layer output
@@ -188,7 +256,7 @@ int oda_recall_score(const float* h_prev, const float* emb, const void* h_local,
  *      e.g. CUDA Graphs) ----------------------------------------------------------------
  * The graph runs, per launch: Local (with commit) at every layer; the recall head on the last
  * layer's Local output; then, inside a conditional IF node that the recall head opens only
- * when some sequence is gated, Full (with gated commit) at every layer not marked local-only.
+ * when some sequence is gated, Full (with gated commit) at every layer.
  * All pointers are captured at creation: the caller refreshes the buffers' contents (seq_lens
  * advanced by one, new q/k/v, new embedding) between launches. */
 typedef struct oda_step_graph oda_step_graph;
@@ -208,8 +276,16 @@ typedef struct {
   const void* const* v_full;
   void* const* out;                    /* [num_layers] fp32 [batch][Hq][128]: selected out   */
   float* const* lse;                   /* nullable; else [num_layers] fp32 [batch][Hq]       */
-  const int32_t* local_only;           /* nullable host int32 [num_layers]: 1 = the layer never
-                                          recomputes with Full (hybrid backbones)           */
+  const int32_t* local_layers;         /* nullable host int32 [num_layers]; per-layer access
+                                          range of the Local attempt ([ODA] 개발자 관점, hybrid
+                                          backbones restrict only some layers to Local):
+                                          non-zero = sink + window, 0 = the layer attends its
+                                          whole history in the attempt too. NULL = every layer
+                                          restricted. The Full recompute attends everything. */
+  const int32_t* sinks;                /* nullable host int32 [num_layers]: per-layer s (>= 0),
+                                          overriding `sink`                                  */
+  const int32_t* windows;              /* nullable host int32 [num_layers]: per-layer w (>= 1),
+                                          overriding `window`                                */
   const float* h_prev;                 /* fp32 [batch][Hq*128], read by the recall head      */
   const float* emb;                    /* fp32 [batch][Hq*128]                               */
   const float* w1;                     /* recall head, as in oda_recall_score                */
@@ -228,9 +304,15 @@ typedef struct {
   int32_t timing_events;               /* 1: event-record nodes at phase boundaries          */
   int32_t phases;                      /* 0 = whole step; else a mask of ODA_PHASE_* (a step
                                           without recall or Full is for measurement only)   */
+  int32_t gate_source;                 /* ODA_GATE_RECALL: the recall head decides;
+                                          ODA_GATE_RANDOM: oda_gate_schedule on gate_u, rho
+                                          (the recall head does not run; q_out untouched)    */
+  const float* gate_u;                 /* RANDOM: device fp32 [batch], refreshed per step    */
+  float rho;                           /* RANDOM: Full-call rate in [0, 1]                   */
 } oda_step_desc;
 
 enum { ODA_PHASE_LOCAL = 1, ODA_PHASE_RECALL = 2, ODA_PHASE_FULL = 4 };
+enum { ODA_GATE_RECALL = 0, ODA_GATE_RANDOM = 1 };
 
 int oda_step_graph_create(const oda_step_desc* desc, void* stream, oda_step_graph** graph);
 int oda_step_graph_launch(oda_step_graph* graph, void* stream);

@@ -30,8 +30,9 @@ extern "C" const char* oda_status_string(int code) {
     case ODA_DEV_BAD_LEN: return "ODA_DEV_BAD_LEN";
     case ODA_DEV_BAD_KEEP_LIST: return "ODA_DEV_BAD_KEEP_LIST";
     case ODA_DEV_TIMEOUT: return "ODA_DEV_TIMEOUT";
+    case ODA_DEV_BAD_DA: return "ODA_DEV_BAD_DA";
     default: return "ODA_UNKNOWN_STATUS";
   }
 }
 
-extern "C" int oda_version(void) { return 100; }
+extern "C" int oda_version(void) { return 101; }

@@ -232,10 +232,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   for (int b = tid; b < B; b += kThreads) {
     const SeqPlan sp = make_plan(p.plan, b);
     pre[b + 1] = sp.npages * Hkv;
-    if (c == 0) {
-      if (sp.bad_len) report(p.status, ODA_DEV_BAD_LEN);
-      if (sp.bad_keep) report(p.status, ODA_DEV_BAD_KEEP_LIST);
-    }
+    if (c == 0 && sp.err != 0) report(p.status, sp.err);
   }
   __syncthreads();
   __shared__ int s_align;  // CTA-count granularity that keeps shares inside one (b, g)
@@ -556,9 +553,8 @@ __global__ void visible_mask_kernel(PlanArgs a, uint8_t* mask, int max_tokens, i
   for (int i = threadIdx.x; i < max_tokens; i += blockDim.x) row[i] = 0;
   __syncthreads();
   const SeqPlan sp = make_plan(a, b);
-  if (sp.bad_len) report(status, ODA_DEV_BAD_LEN);
-  if (sp.bad_keep) report(status, ODA_DEV_BAD_KEEP_LIST);
-  if (sp.skip || sp.bad_len || sp.bad_keep) return;
+  if (sp.err != 0) report(status, sp.err);
+  if (sp.skip || sp.err != 0) return;
   for (int idx = threadIdx.x; idx < sp.npages * kPage; idx += blockDim.x) {
     const int j = idx / kPage, r = idx % kPage;
     const PageRef pr = page_ref(a, sp, b, j);
@@ -675,24 +671,79 @@ static cudaError_t launch_decode_kernel(const DecodeParams& p, int grid, size_t 
   return cudaLaunchKernelEx(&cfg, decode_kernel<G>, p);
 }
 
-int launch_decode(const oda_kv* kv, int mode, const void* q, int hq, int sink, int window,
-                  float scale, const int32_t* gate, const int32_t* keep_blocks,
-                  const int32_t* keep_counts, int max_keep, const void* k_new,
-                  const void* v_new, void* out, int out_dtype, float* lse, void* ws,
-                  size_t ws_bytes, void* stream, int pdl, int wait_first) {
+int check_visibility(const oda_kv* kv, const oda_visibility* v) {
+  if (v == nullptr) return ODA_ERR_INVALID_ARG;
+  switch (v->mode) {
+    case ODA_MODE_LOCAL:
+      return (v->sink < 0 || v->window < 1) ? ODA_ERR_INVALID_ARG : ODA_OK;
+    case ODA_MODE_FULL:
+      return ODA_OK;
+    case ODA_MODE_KEEP:
+      return (v->keep_blocks == nullptr || v->keep_counts == nullptr || v->max_keep < 0 ||
+              v->max_keep > kv->max_blocks_per_seq)
+                 ? ODA_ERR_INVALID_ARG
+                 : ODA_OK;
+    case ODA_MODE_DA:
+      return (v->da_modes == nullptr || v->da_focus_offsets == nullptr || v->da_focus_len < 1 ||
+              v->da_recent < 1 || v->da_local_len < 1)
+                 ? ODA_ERR_INVALID_ARG
+                 : ODA_OK;
+    case ODA_MODE_SHARD:
+      return (v->pos_lo < 0 || v->pos_hi <= v->pos_lo || v->pos_lo % kPage != 0 ||
+              v->pos_hi % kPage != 0)
+                 ? ODA_ERR_INVALID_ARG
+                 : ODA_OK;
+    default:
+      return ODA_ERR_INVALID_ARG;
+  }
+}
+
+static PlanArgs plan_args(const oda_kv* kv, const oda_visibility& v) {
+  PlanArgs a;
+  a.seq_lens = kv->seq_lens;
+  a.block_table = kv->block_table;
+  a.max_blocks = kv->max_blocks_per_seq;
+  a.num_blocks = kv->num_blocks;
+  a.mode = v.mode;
+  a.sink = v.sink;
+  a.window = v.window;
+  a.gate = (v.mode == ODA_MODE_FULL || v.mode == ODA_MODE_SHARD) ? v.gate : nullptr;
+  a.keep_blocks = v.keep_blocks;
+  a.keep_counts = v.keep_counts;
+  a.max_keep = v.max_keep;
+  a.da_modes = v.da_modes;
+  a.da_offsets = v.da_focus_offsets;
+  a.da_focus_len = v.da_focus_len;
+  a.da_recent = v.da_recent;
+  a.da_local_len = v.da_local_len;
+  a.pos_lo = v.pos_lo;
+  a.pos_hi = v.pos_hi;
+  return a;
+}
+
+oda_visibility visibility(int mode) {
+  oda_visibility v = {};
+  v.mode = mode;
+  v.window = 1;
+  return v;
+}
+
+int launch_decode(const oda_kv* kv, const oda_visibility& vis, const void* q, int hq,
+                  float scale, const void* k_new, const void* v_new, void* out, int out_dtype,
+                  float* lse, void* ws, size_t ws_bytes, void* stream, int pdl, int wait_first) {
   int rc = check_kv(kv);
   if (rc != ODA_OK) return rc;
+  if ((rc = check_visibility(kv, &vis)) != ODA_OK) return rc;
   int G = 0;
   if ((rc = group_of(kv, hq, &G)) != ODA_OK) return rc;
   if (out_dtype != ODA_F32 && out_dtype != ODA_BF16) return ODA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return ODA_ERR_INVALID_ARG;
   if ((k_new == nullptr) != (v_new == nullptr)) return ODA_ERR_INVALID_ARG;
+  if (k_new != nullptr && (vis.mode == ODA_MODE_KEEP || vis.mode == ODA_MODE_DA))
+    return ODA_ERR_INVALID_ARG;  // a kept set need not hold slot t
   if (kv->batch == 0) return ODA_OK;
   if (q == nullptr || out == nullptr || ws == nullptr) return ODA_ERR_INVALID_ARG;
   if (!aligned16(q) || (k_new && (!aligned16(k_new) || !aligned16(v_new))))
-    return ODA_ERR_INVALID_ARG;
-  if (mode == ODA_MODE_KEEP && (keep_blocks == nullptr || keep_counts == nullptr || max_keep < 0 ||
-                                max_keep > kv->max_blocks_per_seq))
     return ODA_ERR_INVALID_ARG;
   DeviceInfo di;
   if ((rc = current_device_info(&di)) != ODA_OK) return rc;
@@ -701,17 +752,7 @@ int launch_decode(const oda_kv* kv, int mode, const void* q, int hq, int sink, i
   if (ws_bytes < wl.total) return ODA_ERR_WORKSPACE_TOO_SMALL;
 
   DecodeParams p;
-  p.plan.seq_lens = kv->seq_lens;
-  p.plan.block_table = kv->block_table;
-  p.plan.max_blocks = kv->max_blocks_per_seq;
-  p.plan.num_blocks = kv->num_blocks;
-  p.plan.mode = mode;
-  p.plan.sink = sink;
-  p.plan.window = window;
-  p.plan.gate = gate;
-  p.plan.keep_blocks = keep_blocks;
-  p.plan.keep_counts = keep_counts;
-  p.plan.max_keep = max_keep;
+  p.plan = plan_args(kv, vis);
   p.k_cache = static_cast<const __nv_bfloat16*>(kv->k_cache);
   p.v_cache = static_cast<const __nv_bfloat16*>(kv->v_cache);
   p.k_cache_w = static_cast<__nv_bfloat16*>(kv->k_cache);
@@ -786,22 +827,34 @@ extern "C" int oda_decode_workspace_size(int32_t batch, int32_t num_kv_heads,
   return ODA_OK;
 }
 
+extern "C" int oda_decode(const oda_kv* kv, const oda_visibility* vis, const void* q,
+                          int32_t num_q_heads, float scale, const void* k_new, const void* v_new,
+                          void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                          void* stream) {
+  if (vis == nullptr) return ODA_ERR_INVALID_ARG;
+  return launch_decode(kv, *vis, q, num_q_heads, scale, k_new, v_new, out, out_dtype, lse, ws,
+                       ws_bytes, stream, 0, 0);
+}
+
 extern "C" int oda_decode_local(const oda_kv* kv, const void* q, int32_t num_q_heads,
                                 int32_t sink, int32_t window, float scale, const void* k_new,
                                 const void* v_new, void* out, int32_t out_dtype, float* lse,
                                 void* ws, size_t ws_bytes, void* stream) {
-  if (sink < 0 || window < 1) return ODA_ERR_INVALID_ARG;
-  return launch_decode(kv, ODA_MODE_LOCAL, q, num_q_heads, sink, window, scale, nullptr,
-                       nullptr, nullptr, 0, k_new, v_new, out, out_dtype, lse, ws, ws_bytes,
-                       stream, 0, 0);
+  oda_visibility v = visibility(ODA_MODE_LOCAL);
+  v.sink = sink;
+  v.window = window;
+  return launch_decode(kv, v, q, num_q_heads, scale, k_new, v_new, out, out_dtype, lse, ws,
+                       ws_bytes, stream, 0, 0);
 }
 
 extern "C" int oda_decode_full(const oda_kv* kv, const void* q, int32_t num_q_heads, float scale,
                                const int32_t* gate, const void* k_new, const void* v_new,
                                void* out, int32_t out_dtype, float* lse, void* ws,
                                size_t ws_bytes, void* stream) {
-  return launch_decode(kv, ODA_MODE_FULL, q, num_q_heads, 0, 1, scale, gate, nullptr, nullptr,
-                       0, k_new, v_new, out, out_dtype, lse, ws, ws_bytes, stream, 0, 0);
+  oda_visibility v = visibility(ODA_MODE_FULL);
+  v.gate = gate;
+  return launch_decode(kv, v, q, num_q_heads, scale, k_new, v_new, out, out_dtype, lse, ws,
+                       ws_bytes, stream, 0, 0);
 }
 
 extern "C" int oda_decode_blockmask(const oda_kv* kv, const void* q, int32_t num_q_heads,
@@ -809,39 +862,39 @@ extern "C" int oda_decode_blockmask(const oda_kv* kv, const void* q, int32_t num
                                     const int32_t* keep_counts, int32_t max_keep, void* out,
                                     int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
                                     void* stream) {
-  return launch_decode(kv, ODA_MODE_KEEP, q, num_q_heads, 0, 1, scale, nullptr, keep_blocks,
-                       keep_counts, max_keep, nullptr, nullptr, out, out_dtype, lse, ws,
+  oda_visibility v = visibility(ODA_MODE_KEEP);
+  v.keep_blocks = keep_blocks;
+  v.keep_counts = keep_counts;
+  v.max_keep = max_keep;
+  return launch_decode(kv, v, q, num_q_heads, scale, nullptr, nullptr, out, out_dtype, lse, ws,
                        ws_bytes, stream, 0, 0);
+}
+
+extern "C" int oda_visible_mask_ex(const oda_kv* kv, const oda_visibility* vis, uint8_t* mask,
+                                   int32_t max_tokens, void* stream) {
+  int rc = check_kv(kv);
+  if (rc != ODA_OK) return rc;
+  if ((rc = check_visibility(kv, vis)) != ODA_OK) return rc;
+  if (max_tokens < 0 || (max_tokens > 0 && kv->batch > 0 && mask == nullptr))
+    return ODA_ERR_INVALID_ARG;
+  if (kv->batch == 0 || max_tokens == 0) return ODA_OK;
+  visible_mask_kernel<<<kv->batch, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      plan_args(kv, *vis), mask, max_tokens, kv->dev_status);
+  return cuda_status(cudaGetLastError());
 }
 
 extern "C" int oda_visible_mask(const oda_kv* kv, int32_t mode, int32_t sink, int32_t window,
                                 const int32_t* gate, const int32_t* keep_blocks,
                                 const int32_t* keep_counts, int32_t max_keep, uint8_t* mask,
                                 int32_t max_tokens, void* stream) {
-  int rc = check_kv(kv);
-  if (rc != ODA_OK) return rc;
   if (mode != ODA_MODE_LOCAL && mode != ODA_MODE_FULL && mode != ODA_MODE_KEEP)
     return ODA_ERR_INVALID_ARG;
-  if (mode == ODA_MODE_LOCAL && (sink < 0 || window < 1)) return ODA_ERR_INVALID_ARG;
-  if (mode == ODA_MODE_KEEP && (keep_blocks == nullptr || keep_counts == nullptr || max_keep < 0))
-    return ODA_ERR_INVALID_ARG;
-  if (max_tokens < 0 || (max_tokens > 0 && kv->batch > 0 && mask == nullptr))
-    return ODA_ERR_INVALID_ARG;
-  if (kv->batch == 0 || max_tokens == 0) return ODA_OK;
-  PlanArgs a;
-  a.seq_lens = kv->seq_lens;
-  a.block_table = kv->block_table;
-  a.max_blocks = kv->max_blocks_per_seq;
-  a.num_blocks = kv->num_blocks;
-  a.mode = mode;
-  a.sink = sink;
-  a.window = window;
-  a.gate = mode == ODA_MODE_FULL ? gate : nullptr;
-  a.keep_blocks = keep_blocks;
-  a.keep_counts = keep_counts;
-  a.max_keep = max_keep;
-  visible_mask_kernel<<<kv->batch, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      a, mask, max_tokens, kv->dev_status);
-  return cuda_status(cudaGetLastError());
+  oda_visibility v = visibility(mode);
+  v.sink = sink;
+  v.window = window;
+  v.gate = gate;
+  v.keep_blocks = keep_blocks;
+  v.keep_counts = keep_counts;
+  v.max_keep = max_keep;
+  return oda_visible_mask_ex(kv, &v, mask, max_tokens, stream);
 }
-

@@ -3,7 +3,10 @@
 // Graphs, so that routing needs no host synchronisation).
 //
 // Top-level graph:  [ev0] Local+commit x L  [ev1] recall  [ev2] IF(any gate) [ev3]
-// IF body:          Full+gated commit for every layer not marked local-only
+// (with the random gate source the recall head is replaced by the gate schedule kernel)
+// IF body:          Full+gated commit for every layer
+// A layer outside the Local restriction (hybrid backbones, [ODA] 개발자 관점: the runtime
+// restricts only some layers to Local) attends its whole history in the Local pass as well.
 // The recall kernel sets the IF node's condition from the device on every step (1 iff any
 // sequence is gated), so a step whose sequences are all Local skips the body entirely, and
 // a step with some gated sequences runs Full kernels that skip the ungated ones on-device.
@@ -50,6 +53,9 @@ int record_event_node(oda_step_graph* g, int i) {
   return ODA_OK;
 }
 
+int layer_sink(const oda_step_desc* d, int l) { return d->sinks ? d->sinks[l] : d->sink; }
+int layer_window(const oda_step_desc* d, int l) { return d->windows ? d->windows[l] : d->window; }
+
 int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditionalHandle cond) {
   const int L = d->num_layers;
   const int phases = d->phases ? d->phases : (ODA_PHASE_LOCAL | ODA_PHASE_RECALL | ODA_PHASE_FULL);
@@ -60,9 +66,11 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
   // may start while its predecessor finishes (see the kernels for what they do before
   // waiting). Kernels next to a timing-event node keep ordinary launches.
   for (int l = 0; l < L && (phases & ODA_PHASE_LOCAL); ++l) {
-    if (d->sink < 0 || d->window < 1) return ODA_ERR_INVALID_ARG;
-    rc = oda::launch_decode(&d->layers[l], ODA_MODE_LOCAL, d->q_local[l], d->num_q_heads,
-                            d->sink, d->window, d->scale, nullptr, nullptr, nullptr, 0,
+    const bool restricted = d->local_layers == nullptr || d->local_layers[l] != 0;
+    oda_visibility vis = oda::visibility(restricted ? ODA_MODE_LOCAL : ODA_MODE_FULL);
+    vis.sink = layer_sink(d, l);
+    vis.window = layer_window(d, l);
+    rc = oda::launch_decode(&d->layers[l], vis, d->q_local[l], d->num_q_heads, d->scale,
                             d->k_local[l], d->v_local[l], d->out[l], ODA_F32,
                             d->lse ? d->lse[l] : nullptr, d->decode_ws, d->decode_ws_bytes,
                             g->cap, l > 0 ? 1 : 0, 0);
@@ -75,11 +83,17 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
         if ((rc = record_event_node(g, i)) != ODA_OK) return rc;
     return ODA_OK;
   }
-  const int hidden = d->num_q_heads * d->layers[0].head_dim;
-  rc = oda::launch_recall(d->h_prev, d->emb, d->out[L - 1], ODA_F32, d->layers[0].batch, hidden,
-                          d->mlp, d->w1, d->b1, d->w2, d->b2, d->theta, d->q_out, d->gate_out,
-                          d->full_count, d->use_conditional ? (unsigned long long)cond : 0ull,
-                          d->recall_ws, d->recall_ws_bytes, g->cap, g->timing ? 0 : 1);
+  const unsigned long long cond_u64 = d->use_conditional ? (unsigned long long)cond : 0ull;
+  if (d->gate_source == ODA_GATE_RANDOM) {
+    rc = oda::launch_gate_schedule(d->gate_u, d->layers[0].batch, d->rho, d->gate_out,
+                                   d->full_count, cond_u64, g->cap);
+  } else {
+    const int hidden = d->num_q_heads * d->layers[0].head_dim;
+    rc = oda::launch_recall(d->h_prev, d->emb, d->out[L - 1], ODA_F32, d->layers[0].batch,
+                            hidden, d->mlp, d->w1, d->b1, d->w2, d->b2, d->theta, d->q_out,
+                            d->gate_out, d->full_count, cond_u64, d->recall_ws,
+                            d->recall_ws_bytes, g->cap, g->timing ? 0 : 1);
+  }
   if (rc != ODA_OK) return rc;
   if (g->timing && (rc = record_event_node(g, 2)) != ODA_OK) return rc;
 
@@ -112,21 +126,20 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
       return ODA_ERR_CUDA;
     full_stream = g->cap_body;
   }
-  bool first_full = true;
   for (int l = 0; l < L; ++l) {
-    if (d->local_only != nullptr && d->local_only[l]) continue;
     // The first Full kernel reads the gate the recall head just wrote: inside the IF body it
     // is the body's first node; without the IF node it waits for the recall head at once.
     int pdl = 1, wait_first = 0;
-    if (first_full) {
+    if (l == 0) {
       pdl = (!d->use_conditional && !g->timing) ? 1 : 0;
       wait_first = 1;
     }
-    rc = oda::launch_decode(&d->layers[l], ODA_MODE_FULL, d->q_full[l], d->num_q_heads, 0, 1,
-                            d->scale, d->gate_out, nullptr, nullptr, 0, d->k_full[l],
-                            d->v_full[l], d->out[l], ODA_F32, d->lse ? d->lse[l] : nullptr,
+    oda_visibility vis = oda::visibility(ODA_MODE_FULL);
+    vis.gate = d->gate_out;
+    rc = oda::launch_decode(&d->layers[l], vis, d->q_full[l], d->num_q_heads, d->scale,
+                            d->k_full[l], d->v_full[l], d->out[l], ODA_F32,
+                            d->lse ? d->lse[l] : nullptr,
                             d->decode_ws, d->decode_ws_bytes, full_stream, pdl, wait_first);
-    first_full = false;
     if (rc != ODA_OK) break;
   }
   if (d->use_conditional) {
@@ -153,6 +166,13 @@ int check_desc(const oda_step_desc* d) {
       return ODA_ERR_INVALID_ARG;
   }
   if (k0.batch < 1) return ODA_ERR_INVALID_ARG;
+  for (int l = 0; l < d->num_layers; ++l)
+    if (layer_sink(d, l) < 0 || layer_window(d, l) < 1) return ODA_ERR_INVALID_ARG;
+  if (d->gate_source != ODA_GATE_RECALL && d->gate_source != ODA_GATE_RANDOM)
+    return ODA_ERR_INVALID_ARG;
+  if (d->gate_source == ODA_GATE_RANDOM &&
+      (d->gate_u == nullptr || !(d->rho >= 0.f && d->rho <= 1.f)))
+    return ODA_ERR_INVALID_ARG;
   return ODA_OK;
 }
 

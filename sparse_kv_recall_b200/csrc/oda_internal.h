@@ -18,11 +18,15 @@ int prepare_decode_kernels();
 // Decode launch with optional programmatic dependent launch: pdl = 1 lets the kernel start
 // while the previous kernel of the stream finishes; wait_first = 1 makes it wait for that
 // kernel before reading anything (needed when the previous kernel writes the gate).
-int launch_decode(const oda_kv* kv, int mode, const void* q, int hq, int sink, int window,
-                  float scale, const int32_t* gate, const int32_t* keep_blocks,
-                  const int32_t* keep_counts, int max_keep, const void* k_new,
-                  const void* v_new, void* out, int out_dtype, float* lse, void* ws,
-                  size_t ws_bytes, void* stream, int pdl, int wait_first);
+int launch_decode(const oda_kv* kv, const oda_visibility& vis, const void* q, int hq,
+                  float scale, const void* k_new, const void* v_new, void* out, int out_dtype,
+                  float* lse, void* ws, size_t ws_bytes, void* stream, int pdl, int wait_first);
+
+// A visibility rule with every field zero but `mode` (and window = 1).
+oda_visibility visibility(int mode);
+
+// Host checks of a visibility rule against the cache it is applied to.
+int check_visibility(const oda_kv* kv, const oda_visibility* v);
 
 // oda_kv checks shared by every entry point (ODA_OK or an ODA_ERR_* code).
 int check_kv(const oda_kv* kv);
@@ -37,5 +41,10 @@ int launch_recall(const float* h_prev, const float* emb, const void* h_local, in
                   const float* w2, float b2, float theta, float* q_out, int32_t* gate_out,
                   unsigned long long* full_count, unsigned long long graph_cond_handle,
                   void* ws, size_t ws_bytes, void* stream, int pdl);
+
+// Random gate schedule (gate = u < rho), counters and graph condition as the recall head.
+int launch_gate_schedule(const float* u, int batch, float rho, int32_t* gate_out,
+                         unsigned long long* full_count, unsigned long long graph_cond_handle,
+                         void* stream);
 
 }  // namespace oda

@@ -54,7 +54,8 @@ extern "C" int oda_decode_full_noalloc(const oda_kv* kv, const void* q, int32_t 
   if (cudaMemsetAsync(static_cast<unsigned char*>(ws) + ticket_off, 0, total - ticket_off,
                       static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ODA_ERR_CUDA;
-  return oda::launch_decode(kv, ODA_MODE_FULL, q, num_q_heads, 0, 1, scale, gate, nullptr,
-                            nullptr, 0, k_new, v_new, out, out_dtype, lse, ws,
-                            oda::kStaticWsBytes, stream, 0, 0);
+  oda_visibility vis = oda::visibility(ODA_MODE_FULL);
+  vis.gate = gate;
+  return oda::launch_decode(kv, vis, q, num_q_heads, scale, k_new, v_new, out, out_dtype, lse,
+                            ws, oda::kStaticWsBytes, stream, 0, 0);
 }

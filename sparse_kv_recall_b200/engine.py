@@ -38,6 +38,7 @@ class StagingLayout:
             off += (nbytes + _ALIGN - 1) // _ALIGN * _ALIGN
 
         add("seq_lens", 4 * batch)
+        add("gate_u", 4 * batch)
         add("emb", 4 * batch * hidden)
         for path in ("local", "full"):
             for l in range(layers):
@@ -54,6 +55,8 @@ class StagingLayout:
             raw = buf[off:off + nb]
             if name == "seq_lens":
                 v[name] = raw.view(torch.int32)
+            elif name == "gate_u":
+                v[name] = raw.view(torch.float32)
             elif name == "emb":
                 v[name] = raw.view(torch.float32).view(B, D)
             elif name.startswith("q_"):
@@ -72,7 +75,9 @@ class OdaEngine:
     def __init__(self, k_caches: Sequence[torch.Tensor], v_caches: Sequence[torch.Tensor],
                  block_table: torch.Tensor, num_q_heads: int, recall, theta: float, *,
                  sink: int = 4, window: int = 2048, use_conditional: bool = True,
-                 timing: bool = False, local_only: Optional[Sequence[int]] = None,
+                 timing: bool = False, local_layers: Optional[Sequence[int]] = None,
+                 sinks: Optional[Sequence[int]] = None, windows: Optional[Sequence[int]] = None,
+                 random_rho: Optional[float] = None,
                  with_lse: bool = False, with_stats: bool = True, phases: int = 0):
         self.L = len(k_caches)
         self.B = block_table.shape[0]
@@ -85,7 +90,8 @@ class OdaEngine:
         self.w1, self.b1, self.w2, self.b2 = recall
         self.use_conditional, self.timing = use_conditional, timing
         self.phases = phases
-        self.local_only = local_only
+        self.local_layers, self.sinks, self.windows = local_layers, sinks, windows
+        self.random_rho = random_rho   # not None: random gate schedule at this rate
         dev = block_table.device
         self.layout = StagingLayout(self.L, self.B, self.hq, self.hkv, self.hidden)
         self.staging = torch.zeros(self.layout.nbytes, dtype=torch.uint8, device=dev)
@@ -130,7 +136,10 @@ class OdaEngine:
                 names("q_full"), names("k_full"), names("v_full"),
                 self._layer_out(parity), self.h[parity], v["emb"], self.w1, self.b1, self.w2,
                 self.b2, self.theta, self.q_out, self.gate, self.decode_ws, self.recall_ws,
-                full_count=self.full_count, lse=self.lse, local_only=self.local_only,
+                full_count=self.full_count, lse=self.lse, local_layers=self.local_layers,
+                sinks=self.sinks, windows=self.windows,
+                gate_u=v["gate_u"] if self.random_rho is not None else None,
+                rho=self.random_rho or 0.0,
                 use_conditional=self.use_conditional, timing_events=self.timing,
                 phases=self.phases))
 
@@ -161,6 +170,8 @@ def fill_staging(views: dict, step_inputs, seq_lens: Sequence[int]):
     """Copy one step's inputs (oda_synth.StepInputs or any object with the same fields) into
     staging views (of a device staging buffer or of one slot of a pool)."""
     views["seq_lens"].copy_(torch.as_tensor(seq_lens, dtype=torch.int32))
+    if getattr(step_inputs, "gate_u", None) is not None:
+        views["gate_u"].copy_(step_inputs.gate_u)
     views["emb"].copy_(step_inputs.emb)
     for path in ("local", "full"):
         for kind in ("q", "k", "v"):

@@ -24,17 +24,25 @@ ODA_DEV_BAD_BLOCK = 1
 ODA_DEV_BAD_LEN = 2
 ODA_DEV_BAD_KEEP_LIST = 3
 ODA_DEV_TIMEOUT = 4
+ODA_DEV_BAD_DA = 5
 ODA_F32 = 0
 ODA_BF16 = 1
 ODA_MODE_LOCAL = 0
 ODA_MODE_FULL = 1
 ODA_MODE_KEEP = 2
+ODA_MODE_DA = 3
+ODA_MODE_SHARD = 4
+ODA_DA_GLOBAL = 0
+ODA_DA_FOCUS = 1
+ODA_DA_LOCAL = 2
 ODA_STAT_ROWS = 0
 ODA_STAT_PAGES = 1
 ODA_STATS_LEN = 2
 ODA_PHASE_LOCAL = 1
 ODA_PHASE_RECALL = 2
 ODA_PHASE_FULL = 4
+ODA_GATE_RECALL = 0
+ODA_GATE_RANDOM = 1
 
 
 class OdaError(RuntimeError):
@@ -57,6 +65,17 @@ class oda_kv(ctypes.Structure):
     ]
 
 
+class oda_visibility(ctypes.Structure):
+    _fields_ = [
+        ("mode", ctypes.c_int32), ("sink", ctypes.c_int32), ("window", ctypes.c_int32),
+        ("gate", ctypes.c_void_p), ("keep_blocks", ctypes.c_void_p),
+        ("keep_counts", ctypes.c_void_p), ("max_keep", ctypes.c_int32),
+        ("da_modes", ctypes.c_void_p), ("da_focus_offsets", ctypes.c_void_p),
+        ("da_focus_len", ctypes.c_int32), ("da_recent", ctypes.c_int32),
+        ("da_local_len", ctypes.c_int32), ("pos_lo", ctypes.c_int32), ("pos_hi", ctypes.c_int32),
+    ]
+
+
 class oda_step_desc(ctypes.Structure):
     _fields_ = [
         ("num_layers", ctypes.c_int32), ("layers", ctypes.POINTER(oda_kv)),
@@ -66,7 +85,8 @@ class oda_step_desc(ctypes.Structure):
         ("v_local", ctypes.POINTER(ctypes.c_void_p)), ("q_full", ctypes.POINTER(ctypes.c_void_p)),
         ("k_full", ctypes.POINTER(ctypes.c_void_p)), ("v_full", ctypes.POINTER(ctypes.c_void_p)),
         ("out", ctypes.POINTER(ctypes.c_void_p)), ("lse", ctypes.POINTER(ctypes.c_void_p)),
-        ("local_only", ctypes.POINTER(ctypes.c_int32)),
+        ("local_layers", ctypes.POINTER(ctypes.c_int32)), ("sinks", ctypes.POINTER(ctypes.c_int32)),
+        ("windows", ctypes.POINTER(ctypes.c_int32)),
         ("h_prev", ctypes.c_void_p), ("emb", ctypes.c_void_p),
         ("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("w2", ctypes.c_void_p),
         ("b2", ctypes.c_float), ("theta", ctypes.c_float), ("mlp", ctypes.c_int32),
@@ -74,7 +94,8 @@ class oda_step_desc(ctypes.Structure):
         ("decode_ws", ctypes.c_void_p), ("decode_ws_bytes", ctypes.c_size_t),
         ("recall_ws", ctypes.c_void_p), ("recall_ws_bytes", ctypes.c_size_t),
         ("use_conditional", ctypes.c_int32), ("timing_events", ctypes.c_int32),
-        ("phases", ctypes.c_int32),
+        ("phases", ctypes.c_int32), ("gate_source", ctypes.c_int32),
+        ("gate_u", ctypes.c_void_p), ("rho", ctypes.c_float),
     ]
 
 
@@ -84,6 +105,8 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int32
 _F = ctypes.c_float
 _SZ = ctypes.c_size_t
+
+_VIS = ctypes.POINTER(oda_visibility)
 
 _SIGNATURES = {
     "oda_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -97,6 +120,10 @@ _SIGNATURES = {
     "oda_decode_blockmask": (ctypes.c_int, [_KV, _P, _I, _F, _P, _P, _I, _P, _I, _P, _P, _SZ, _P]),
     "oda_decode_full_noalloc": (ctypes.c_int, [_KV, _P, _I, _F, _P, _P, _P, _P, _I, _P, _P]),
     "oda_visible_mask": (ctypes.c_int, [_KV, _I, _I, _I, _P, _P, _P, _I, _P, _I, _P]),
+    "oda_decode": (ctypes.c_int, [_KV, _VIS, _P, _I, _F, _P, _P, _P, _I, _P, _P, _SZ, _P]),
+    "oda_visible_mask_ex": (ctypes.c_int, [_KV, _VIS, _P, _I, _P]),
+    "oda_merge_partials": (ctypes.c_int, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _P]),
+    "oda_gate_schedule": (ctypes.c_int, [_P, _I, _F, _P, _P, ctypes.c_ulonglong, _P]),
     "oda_recall_score": (ctypes.c_int, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _F, _F, _P, _P, _P,
                                         ctypes.c_ulonglong, _P, _SZ, _P]),
     "oda_step_graph_create": (ctypes.c_int, [ctypes.POINTER(oda_step_desc), _P,
@@ -174,7 +201,7 @@ def make_kv(k_cache, v_cache, block_table, seq_lens, dev_status=None, stats=None
     """oda_kv for bf16 caches [num_blocks][Hkv][16][128], int32 block_table [B][maxb] and
     int32 seq_lens [B] (tokens including the current one)."""
     nb, hkv, bs, d = k_cache.shape
-    return oda_kv(
+    kv = oda_kv(
         k_cache=_ptr(k_cache, torch.bfloat16, "k_cache"),
         v_cache=_ptr(v_cache, torch.bfloat16, "v_cache"),
         block_table=_ptr(block_table, torch.int32, "block_table"),
@@ -183,6 +210,8 @@ def make_kv(k_cache, v_cache, block_table, seq_lens, dev_status=None, stats=None
         max_blocks_per_seq=block_table.shape[1], num_blocks=nb,
         dev_status=_ptr(dev_status, torch.int32, "dev_status"),
         stats=_ptr(stats, torch.int64, "stats"))
+    kv._refs = (k_cache, v_cache, block_table, seq_lens, dev_status, stats)
+    return kv
 
 
 def oda_decode_workspace_size(batch: int, num_kv_heads: int, num_q_heads: int) -> int:
@@ -255,6 +284,59 @@ def oda_visible_mask(kv: oda_kv, mode: int, mask, sink: int = 0, window: int = 1
         "oda_visible_mask")
 
 
+def da_visibility(modes, focus_offsets, focus_len: int = 32768, recent: int = 2048,
+                  local_len: int = 4096) -> oda_visibility:
+    """Declarative-Attention rule: one declared mode per sequence (int32 [B], ODA_DA_*) and
+    the focused region's first position (int32 [B]), compiled into page runs on the device."""
+    v = oda_visibility(mode=ODA_MODE_DA, window=1,
+                       da_modes=_ptr(modes, torch.int32, "modes"),
+                       da_focus_offsets=_ptr(focus_offsets, torch.int32, "focus_offsets"),
+                       da_focus_len=focus_len, da_recent=recent, da_local_len=local_len)
+    v._refs = (modes, focus_offsets)      # the rule holds device pointers: keep them alive
+    return v
+
+
+def shard_visibility(pos_lo: int, pos_hi: int, gate=None) -> oda_visibility:
+    """Positions [pos_lo, pos_hi) of 0..t (page-aligned): one GPU's part of a Full pass."""
+    v = oda_visibility(mode=ODA_MODE_SHARD, window=1, gate=_ptr(gate, torch.int32, "gate"),
+                       pos_lo=int(pos_lo), pos_hi=int(pos_hi))
+    v._refs = (gate,)
+    return v
+
+
+def oda_decode(kv: oda_kv, vis: oda_visibility, q, scale: float, out, ws, k_new=None,
+               v_new=None, lse=None, stream=None):
+    """Decode attention under any visibility rule (oda_visibility)."""
+    _check(load().oda_decode(
+        ctypes.byref(kv), ctypes.byref(vis), _ptr(q, torch.bfloat16, "q"), q.shape[1], scale,
+        _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        _ptr(out, None, "out"), _out_dtype(out), _ptr(lse, torch.float32, "lse"),
+        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)), "oda_decode")
+
+
+def oda_visible_mask_ex(kv: oda_kv, vis: oda_visibility, mask, stream=None):
+    _check(load().oda_visible_mask_ex(ctypes.byref(kv), ctypes.byref(vis),
+                                      _ptr(mask, torch.uint8, "mask"), mask.shape[1],
+                                      _stream(stream)), "oda_visible_mask_ex")
+
+
+def oda_merge_partials(o_parts, lse_parts, out, gate=None, lse=None, stream=None):
+    """o_parts fp32 [R][B][Hq][128], lse_parts fp32 [R][B][Hq] -> out [B][Hq][128]."""
+    R, B, Hq, _ = o_parts.shape
+    _check(load().oda_merge_partials(
+        _ptr(o_parts, torch.float32, "o_parts"), _ptr(lse_parts, torch.float32, "lse_parts"),
+        R, B, Hq, _ptr(gate, torch.int32, "gate"), _ptr(out, None, "out"), _out_dtype(out),
+        _ptr(lse, torch.float32, "lse"), _stream(stream)), "oda_merge_partials")
+
+
+def oda_gate_schedule(u, rho: float, gate_out, full_count=None, graph_cond_handle: int = 0,
+                      stream=None):
+    _check(load().oda_gate_schedule(
+        _ptr(u, torch.float32, "u"), u.shape[0], float(rho), _ptr(gate_out, torch.int32, "gate_out"),
+        _ptr(full_count, torch.int64, "full_count"), int(graph_cond_handle), _stream(stream)),
+        "oda_gate_schedule")
+
+
 def oda_recall_score(h_prev, emb, h_local, w1, b1, w2, b2: float, theta: float, q_out, gate_out,
                      ws, full_count=None, graph_cond_handle: int = 0, stream=None):
     batch, hidden = h_prev.shape
@@ -282,8 +364,9 @@ class StepGraph:
     def __init__(self, kvs: Sequence[oda_kv], num_q_heads: int, sink: int, window: int,
                  scale: float, q_local, k_local, v_local, q_full, k_full, v_full, out,
                  h_prev, emb, w1, b1, w2, b2: float, theta: float, q_out, gate_out,
-                 decode_ws, recall_ws, full_count=None, lse=None, local_only=None,
-                 use_conditional: bool = True, timing_events: bool = False, phases: int = 0):
+                 decode_ws, recall_ws, full_count=None, lse=None, local_layers=None,
+                 sinks=None, windows=None, use_conditional: bool = True,
+                 timing_events: bool = False, phases: int = 0, gate_u=None, rho: float = 0.0):
         L = len(kvs)
         self._keep = []
         layers = (oda_kv * L)(*kvs)
@@ -293,8 +376,17 @@ class StepGraph:
                                                    (k_full, "k_full"), (v_full, "v_full"))]
         outs = _ptr_array(out, torch.float32, "out")
         lses = _ptr_array(lse, torch.float32, "lse") if lse is not None else None
-        lo = (ctypes.c_int32 * L)(*[int(x) for x in local_only]) if local_only is not None else None
-        self._keep += [layers, outs, lses, lo] + arrs
+        def ints(xs, name):
+            if xs is None:
+                return None
+            if len(xs) != L:
+                raise ValueError("%s: %d entries for %d layers" % (name, len(xs), L))
+            return (ctypes.c_int32 * L)(*[int(x) for x in xs])
+
+        ll, sk, wn = ints(local_layers, "local_layers"), ints(sinks, "sinks"), ints(windows, "windows")
+        self._keep += [layers, outs, lses, ll, sk, wn] + arrs
+        ip = ctypes.POINTER(ctypes.c_int32)
+        icast = lambda a: ctypes.cast(a, ip) if a is not None else None
         vp = ctypes.POINTER(ctypes.c_void_p)
         d = oda_step_desc(
             num_layers=L, layers=ctypes.cast(layers, ctypes.POINTER(oda_kv)),
@@ -303,7 +395,7 @@ class StepGraph:
             v_local=ctypes.cast(arrs[2], vp), q_full=ctypes.cast(arrs[3], vp),
             k_full=ctypes.cast(arrs[4], vp), v_full=ctypes.cast(arrs[5], vp),
             out=ctypes.cast(outs, vp), lse=ctypes.cast(lses, vp) if lses is not None else None,
-            local_only=ctypes.cast(lo, ctypes.POINTER(ctypes.c_int32)) if lo is not None else None,
+            local_layers=icast(ll), sinks=icast(sk), windows=icast(wn),
             h_prev=_ptr(h_prev, torch.float32, "h_prev"), emb=_ptr(emb, torch.float32, "emb"),
             w1=_ptr(w1, torch.float32, "w1"), b1=_ptr(b1, torch.float32, "b1"),
             w2=_ptr(w2, torch.float32, "w2"), b2=float(b2), theta=float(theta), mlp=w1.shape[1],
@@ -314,7 +406,9 @@ class StepGraph:
             recall_ws=_ptr(recall_ws, None, "recall_ws"),
             recall_ws_bytes=recall_ws.numel() * recall_ws.element_size(),
             use_conditional=int(bool(use_conditional)), timing_events=int(bool(timing_events)),
-            phases=int(phases))
+            phases=int(phases),
+            gate_source=ODA_GATE_RANDOM if gate_u is not None else ODA_GATE_RECALL,
+            gate_u=_ptr(gate_u, torch.float32, "gate_u"), rho=float(rho))
         self._desc = d
         h = ctypes.c_void_p(0)
         _check(load().oda_step_graph_create(ctypes.byref(d), None, ctypes.byref(h)),

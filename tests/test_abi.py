@@ -36,10 +36,11 @@ def test_status_strings_and_version(lib):
     for code, name in [(0, "ODA_OK"), (-1, "ODA_ERR_INVALID_ARG"), (-2, "ODA_ERR_UNSUPPORTED_SHAPE"),
                        (-3, "ODA_ERR_WORKSPACE_TOO_SMALL"), (-4, "ODA_ERR_CUDA"),
                        (-5, "ODA_ERR_NOT_IMPLEMENTED"), (1, "ODA_DEV_BAD_BLOCK"),
-                       (2, "ODA_DEV_BAD_LEN"), (3, "ODA_DEV_BAD_KEEP_LIST"), (4, "ODA_DEV_TIMEOUT")]:
+                       (2, "ODA_DEV_BAD_LEN"), (3, "ODA_DEV_BAD_KEEP_LIST"), (4, "ODA_DEV_TIMEOUT"),
+                       (5, "ODA_DEV_BAD_DA")]:
         assert oda.oda_status_string(code) == name
     assert oda.oda_status_string(99) == "ODA_UNKNOWN_STATUS"
-    assert oda.oda_version() == 100
+    assert oda.oda_version() == 101
 
 
 def _kv(**kw):
@@ -117,3 +118,43 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(oda, "_LIB_PATH", str(tmp_path / "liboda.so"))
     with pytest.raises(RuntimeError, match="liboda.so not found"):
         oda.load()
+
+
+def _decode(lib, vis, kv=None, k_new=None, v_new=None):
+    kv = kv or _kv()
+    return lib.oda_decode(ctypes.byref(kv), ctypes.byref(vis) if vis is not None else None,
+                          0x70000, 16, 0.088, k_new, v_new, 0x50000, 0, None, 0x60000, 1 << 40,
+                          None)
+
+
+def test_visibility_argument_checks(lib):
+    I, OK = oda.ODA_ERR_INVALID_ARG, oda.ODA_OK
+    V = oda.oda_visibility
+    assert _decode(lib, None) == I
+    assert _decode(lib, V(mode=9, window=1)) == I
+    assert _decode(lib, V(mode=oda.ODA_MODE_LOCAL, sink=4, window=0)) == I
+    assert _decode(lib, V(mode=oda.ODA_MODE_DA, window=1, da_focus_len=16, da_recent=16,
+                          da_local_len=16)) == I                       # no mode array
+    assert _decode(lib, V(mode=oda.ODA_MODE_DA, window=1, da_modes=0x1000, da_focus_offsets=0x2000,
+                          da_focus_len=0, da_recent=16, da_local_len=16)) == I
+    assert _decode(lib, V(mode=oda.ODA_MODE_DA, window=1, da_modes=0x1000, da_focus_offsets=0x2000,
+                          da_focus_len=16, da_recent=16, da_local_len=16),
+                   k_new=0x80000, v_new=0x90000) == I              # DA need not hold slot t
+    for lo, hi in [(-16, 32), (8, 32), (0, 24), (32, 32), (48, 32)]:
+        assert _decode(lib, V(mode=oda.ODA_MODE_SHARD, window=1, pos_lo=lo, pos_hi=hi)) == I
+    assert _decode(lib, V(mode=oda.ODA_MODE_SHARD, window=1, pos_lo=0, pos_hi=32),
+                   kv=_kv(batch=0)) == OK                          # nothing to do
+    assert lib.oda_visible_mask_ex(ctypes.byref(_kv()), None, 0x1000, 10, None) == I
+
+
+def test_merge_and_schedule_argument_checks(lib):
+    I, OK = oda.ODA_ERR_INVALID_ARG, oda.ODA_OK
+    assert lib.oda_merge_partials(0x1000, 0x2000, 0, 1, 16, None, 0x3000, 0, None, None) == I
+    assert lib.oda_merge_partials(0x1000, 0x2000, 65, 1, 16, None, 0x3000, 0, None, None) == I
+    assert lib.oda_merge_partials(0x1000, 0x2000, 2, 1, 16, None, 0x3000, 5, None, None) == I
+    assert lib.oda_merge_partials(None, 0x2000, 2, 1, 16, None, 0x3000, 0, None, None) == I
+    assert lib.oda_merge_partials(0x1000, 0x2000, 2, 0, 16, None, 0x3000, 0, None, None) == OK
+    assert lib.oda_gate_schedule(0x1000, 4, 1.5, 0x2000, None, 0, None) == I
+    assert lib.oda_gate_schedule(0x1000, 4, float("nan"), 0x2000, None, 0, None) == I
+    assert lib.oda_gate_schedule(None, 4, 0.5, 0x2000, None, 0, None) == I
+    assert lib.oda_gate_schedule(0x1000, 0, 0.5, 0x2000, None, 0, None) == OK

@@ -30,13 +30,15 @@ def _logical(bits, bt, caps, hkv, d):
     return out
 
 
-def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02, timing=False):
+def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02, timing=False,
+               **layer_ranges):
     lay = oda_synth.make_layout(w, extra_tokens=steps + 2, device="cuda", lengths=lengths)
     caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
     rw = oda_synth.make_recall_weights(w, device="cuda", std=recall_std)
     eng = OdaEngine([c[0] for c in caches], [c[1] for c in caches], lay.block_table,
                     w.num_q_heads, (rw.w1, rw.b1, rw.w2, rw.b2), theta, sink=w.sink,
-                    window=w.window, use_conditional=use_conditional, timing=timing)
+                    window=w.window, use_conditional=use_conditional, timing=timing,
+                    **layer_ranges)
     h0 = oda_synth.make_h0(w, device="cuda")
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     for e in evs:
@@ -49,7 +51,7 @@ def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02, 
     rec = (rw.w1.double().cpu().numpy(), rw.b1.double().cpu().numpy(),
            rw.w2.double().cpu().numpy(), rw.b2)
     dec = O.OdaDecoder(kh, vh, lengths, h0.double().cpu().numpy(), rec, sink=w.sink,
-                       window=w.window, theta=theta)
+                       window=w.window, theta=theta, **layer_ranges)
     n_gated = 0
     n_phases = 0
     for i in range(steps):
@@ -69,10 +71,15 @@ def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02, 
         inp = {k: [oda_synth.bf16_bits(x) for x in getattr(si, k)]
                for k in ("q_local", "k_local", "v_local", "q_full", "k_full", "v_full")}
         inp["emb"] = si.emb.double().cpu().numpy()
-        ref, _, rq, rg = dec.step(inp, gate_hint=gate)
-        assert np.abs(q - rq).max() <= Q_TOL, (i, q, rq)
-        sure = np.abs(rq - theta) >= Q_TOL
-        assert np.array_equal(gate[sure], rg[sure]), (i, gate, rg)
+        inp["gate_u"] = si.gate_u.cpu().numpy()
+        if layer_ranges.get("random_rho") is not None:
+            ref, _, _, rg = dec.step(inp)
+            assert np.array_equal(gate, rg), (i, gate, rg)   # the schedule decides, exactly
+        else:
+            ref, _, rq, rg = dec.step(inp, gate_hint=gate)
+            assert np.abs(q - rq).max() <= Q_TOL, (i, q, rq)
+            sure = np.abs(rq - theta) >= Q_TOL
+            assert np.array_equal(gate[sure], rg[sure]), (i, gate, rg)
         assert_attn_close(outs, ref, "step %d" % i)
         n_gated += int(gate.sum())
         n_phases += int(gate.any())
@@ -93,6 +100,27 @@ def test_step_graph_matches_oracle_ragged(use_conditional):
                            prefill=300, steps=6, seed=77, sink=4, window=64)
     n = _run_steps(w, [300, 37, 170], 6, theta=0.0, use_conditional=use_conditional)
     assert 0 < n < 18                      # both paths exercised
+
+
+def test_step_graph_per_layer_access_range():
+    """Hybrid backbone: layer 1 is outside the Local restriction (attends its whole history
+    in the Local attempt), layers 0 and 2 have their own sink and window."""
+    w = oda_synth.Workload(name="hybrid", layers=3, batch=3, num_q_heads=16, num_kv_heads=8,
+                           prefill=300, steps=5, seed=81, sink=4, window=64)
+    n = _run_steps(w, [300, 37, 520], 5, theta=0.0, local_layers=[1, 0, 1], sinks=[4, 0, 0],
+                   windows=[64, 64, 17])
+    assert 0 < n < 15
+
+
+@pytest.mark.parametrize("use_conditional", [True, False])
+def test_step_graph_random_gate_schedule(use_conditional):
+    """The random-timing ablation: the recall head is replaced by gate = u < rho on the
+    step's uniform draws; everything downstream (IF node, gated Full, commit) is unchanged."""
+    w = oda_synth.Workload(name="random", layers=2, batch=4, num_q_heads=16, num_kv_heads=8,
+                           prefill=400, steps=6, seed=82, sink=4, window=64)
+    n = _run_steps(w, [400, 90, 1000, 17], 6, theta=0.0, use_conditional=use_conditional,
+                   random_rho=0.4)
+    assert 0 < n < 24
 
 
 def test_step_graph_with_timing_events():
