@@ -33,6 +33,7 @@ _P_EMB = 7
 _P_LENGTHS = 8
 _P_DAMODE = 9
 _P_GATE_U = 10
+_P_GAIN = 11
 
 
 @dataclasses.dataclass(frozen=True)
@@ -237,6 +238,17 @@ def make_recall_weights(w: Workload, device="cpu", std: float = 0.02) -> RecallW
     w2 = torch.randn((w.mlp,), generator=g, dtype=torch.float32) * std
     b1 = torch.zeros((w.mlp,), dtype=torch.float32)
     return RecallWeights(w1=w1.to(device), b1=b1.to(device), w2=w2.to(device), b2=0.0)
+
+
+def make_gains(w: Workload, step: int, device="cpu") -> torch.Tensor:
+    """Synthetic per-sequence gains g_t = log p^F - log p^L of Full over Local (fp32 [B]) for
+    recall-head training: most steps gain almost nothing from Full (N(0, 0.1^2)), about one
+    in five gains a lot (|N(0, 3^2)|), the shape the pages' recall rates imply."""
+    g = _gen(w.seed, _P_GAIN, step)
+    small = torch.randn((w.batch,), generator=g, dtype=torch.float32) * 0.1
+    big = torch.randn((w.batch,), generator=g, dtype=torch.float32).abs() * 3.0
+    pick = torch.rand((w.batch,), generator=g, dtype=torch.float32) < 0.2
+    return torch.where(pick, big, small).to(device)
 
 
 @dataclasses.dataclass

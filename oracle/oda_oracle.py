@@ -209,6 +209,54 @@ def gate(q, theta: float = DEFAULT_THETA):
 
 
 # ----------------------------------------------------------------------------------------
+# Recall-head training objective ([ODA] 핵심 기여 and 접근 방법: the gain of Full over Local
+# g_t = log p^F - log p^L, its cost-adjusted form d_t = g_t - lambda, the signed-log target
+# y_t = sign(d_t) log(1 + |d_t|), and Huber regression with delta = 1 of q_t on y_t).
+# ----------------------------------------------------------------------------------------
+def signed_log_target(gain, lam: float):
+    """y = sign(d) log(1 + |d|) with d = gain - lambda."""
+    d = np.asarray(gain, dtype=np.float64) - lam
+    return np.sign(d) * np.log1p(np.abs(d))
+
+
+def huber(r, delta: float = 1.0):
+    """r^2 / 2 for |r| <= delta, delta (|r| - delta / 2) beyond."""
+    r = np.asarray(r, dtype=np.float64)
+    a = np.abs(r)
+    return np.where(a <= delta, 0.5 * r * r, delta * (a - 0.5 * delta))
+
+
+def gelu_grad(z):
+    """d/dz of z Phi(z): Phi(z) + z phi(z)."""
+    z = np.asarray(z, dtype=np.float64)
+    erf = np.vectorize(math.erf, otypes=[np.float64])
+    return 0.5 * (1.0 + erf(z / math.sqrt(2.0))) + z * np.exp(-0.5 * z * z) / math.sqrt(2 * math.pi)
+
+
+def recall_loss_grad(h_prev, emb, h_local, W1, b1, w2, b2, gain, lam: float, delta: float = 1.0):
+    """Mean Huber loss of the recall head over a batch and its gradient with respect to the
+    head's parameters (the backbone is frozen). The pages do not print the reduction; the
+    batch mean is taken. Returns (loss, q [B], dW1 [3D][M], db1 [M], dw2 [M], db2)."""
+    x = np.concatenate([np.asarray(h_prev, np.float64), np.asarray(emb, np.float64),
+                        np.asarray(h_local, np.float64)], axis=-1)
+    W1, b1, w2 = (np.asarray(a, np.float64) for a in (W1, b1, w2))
+    z = x @ W1 + b1
+    a = gelu(z)
+    q = a @ w2 + float(b2)
+    y = signed_log_target(gain, lam)
+    r = q - y
+    B = x.shape[0]
+    loss = float(huber(r, delta).sum() / B)
+    dq = np.clip(r, -delta, delta) / B            # d loss / d q_b
+    dw2 = a.T @ dq
+    db2 = float(dq.sum())
+    dz = np.outer(dq, w2) * gelu_grad(z)          # [B][M]
+    db1 = dz.sum(axis=0)
+    dW1 = x.T @ dz
+    return loss, q, dW1, db1, dw2, db2
+
+
+# ----------------------------------------------------------------------------------------
 # Cost model.
 # ----------------------------------------------------------------------------------------
 def attended_tokens(t: int, gated: bool, sink: int = DEFAULT_SINK,

@@ -472,3 +472,76 @@ def test_window_of_one_sees_only_the_new_token():
                 s = float(O.widen_bf16(inp["q_local"][layer][b][h]) @
                           O.widen_bf16(inp["k_local"][layer][b][h // G])) / math.sqrt(wl.head_dim)
                 assert lse[layer, b, h] == pytest.approx(s, abs=1e-12)
+
+
+# ---------------------------------------------------------------- recall-head training objective
+def test_signed_log_target_values():
+    assert O.signed_log_target(0.0, 0.0) == 0.0
+    assert O.signed_log_target(math.e - 1, 0.0) == pytest.approx(1.0, abs=1e-15)
+    assert O.signed_log_target(0.5, 0.5 + math.e ** 2 - 1) == pytest.approx(-2.0, abs=1e-14)
+    d = np.linspace(-5, 5, 41)
+    np.testing.assert_allclose(O.signed_log_target(d, 0.0), -O.signed_log_target(-d, 0.0), atol=0)
+    assert np.all(np.diff(O.signed_log_target(d, 0.0)) > 0)            # strictly increasing
+
+
+def test_huber_closed_forms():
+    assert O.huber(0.5) == 0.125 and O.huber(-0.5) == 0.125
+    assert O.huber(3.0) == 2.5 and O.huber(-3.0) == 2.5                 # 1 * (3 - 1/2)
+    assert O.huber(1.0) == 0.5                                          # both branches meet
+    assert O.huber(4.0, delta=2.0) == 6.0                               # 2 * (4 - 1)
+
+
+def test_gelu_grad_against_central_differences():
+    z = np.linspace(-6, 6, 49)
+    h = 1e-6
+    num = (O.gelu(z + h) - O.gelu(z - h)) / (2 * h)
+    np.testing.assert_allclose(O.gelu_grad(z), num, atol=1e-9)
+    assert O.gelu_grad(0.0) == 0.5
+
+
+def _train_case(B=3, D=3, M=4, seed=11, scale=0.7):
+    r = _rng(seed)
+    hp, em, hl = (r.standard_normal((B, D)) for _ in range(3))
+    W1 = r.standard_normal((3 * D, M)) * scale
+    b1, w2 = r.standard_normal(M) * scale, r.standard_normal(M) * scale
+    gain = np.array([0.05, 8.0, -5.0])[:B]
+    return hp, em, hl, W1, b1, w2, 0.3, gain
+
+
+def test_recall_gradient_against_central_differences():
+    hp, em, hl, W1, b1, w2, b2, gain = _train_case()
+    lam = 0.2
+    loss, q, dW1, db1, dw2, db2 = O.recall_loss_grad(hp, em, hl, W1, b1, w2, b2, gain, lam)
+    # the residuals straddle delta = 1, so both Huber branches are exercised
+    r = q - O.signed_log_target(gain, lam)
+    assert (np.abs(r) < 1).any() and (np.abs(r) > 1).any()
+    f = lambda W1_, b1_, w2_, b2_: O.recall_loss_grad(hp, em, hl, W1_, b1_, w2_, b2_, gain, lam)[0]
+    h = 1e-6
+    for arr, grad in ((W1, dW1), (b1, db1), (w2, dw2)):
+        for idx in np.ndindex(arr.shape):
+            up, dn = arr.copy(), arr.copy()
+            up[idx] += h
+            dn[idx] -= h
+            args_up = [up if x is arr else x for x in (W1, b1, w2)]
+            args_dn = [dn if x is arr else x for x in (W1, b1, w2)]
+            num = (f(*args_up, b2) - f(*args_dn, b2)) / (2 * h)
+            assert abs(num - grad[idx]) < 1e-7, (idx, num, grad[idx])
+    num = (f(W1, b1, w2, b2 + h) - f(W1, b1, w2, b2 - h)) / (2 * h)
+    assert abs(num - db2) < 1e-7
+    # the forward half is the recall head itself
+    np.testing.assert_allclose(q, O.recall_score(hp, em, hl, W1, b1, w2, b2), atol=0)
+
+
+def test_recall_loss_with_silent_head_is_closed_form():
+    """W1 = 0, b1 = 0, w2 = 0: q = b2 for every row, so loss = mean Huber(b2 - y), the only
+    nonzero gradient is db2 = mean clip(b2 - y), and dW1, db1, dw2 vanish."""
+    hp, em, hl, W1, b1, w2, _, gain = _train_case(B=3)
+    W1, b1, w2 = np.zeros_like(W1), np.zeros_like(b1), np.zeros_like(w2)
+    b2, lam = 0.4, 0.0
+    loss, q, dW1, db1, dw2, db2 = O.recall_loss_grad(hp, em, hl, W1, b1, w2, b2, gain, lam)
+    y = [math.copysign(math.log1p(abs(g)), g) for g in gain]
+    assert np.all(q == b2)
+    want = sum(0.5 * (b2 - t) ** 2 if abs(b2 - t) <= 1 else abs(b2 - t) - 0.5 for t in y) / 3
+    assert loss == pytest.approx(want, abs=1e-15)
+    assert db2 == pytest.approx(sum(min(max(b2 - t, -1), 1) for t in y) / 3, abs=1e-15)
+    assert not dW1.any() and not db1.any() and not dw2.any()
