@@ -425,6 +425,43 @@ def cp_emulation(s, w, stream, reps: int = 10):
     return res
 
 
+def run_train_grad(w, dev, stream, batch: int = 8, reps: int = 50):
+    """Recall-head training objective: loss and gradient (oda_recall_loss_grad, three
+    launches) for a batch of `batch` rows at the workload's hidden size, timed over `reps`
+    calls captured in one CUDA graph. Bytes: W1 read once, dW1 written once."""
+    from sparse_kv_recall_b200 import oda
+    wl = oda_synth.scaled(w, batch=batch, name=w.name + "-train")
+    rw = oda_synth.make_recall_weights(wl, device=dev)
+    g = torch.Generator(device=dev).manual_seed(wl.seed)
+    hp, em, hl = (torch.randn(batch, wl.hidden, generator=g, device=dev) for _ in range(3))
+    gain = oda_synth.make_gains(wl, 0, device=dev)
+    ws = torch.zeros(oda.oda_recall_train_workspace_size(batch, wl.hidden, wl.mlp),
+                     dtype=torch.uint8, device=dev)
+    loss, db2 = torch.empty(1, device=dev), torch.empty(1, device=dev)
+    dw1, db1, dw2 = torch.empty_like(rw.w1), torch.empty_like(rw.b1), torch.empty_like(rw.w2)
+    call = lambda: oda.oda_recall_loss_grad(hp, em, hl, rw.w1, rw.b1, rw.w2, rw.b2, gain, 0.5, ws,
+                                            loss, dw1, db1, dw2, db2)
+    call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(reps):
+            call()
+    graph.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    graph.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) / reps * 1e3
+    nbytes = 2 * rw.w1.numel() * 4
+    del graph
+    return {"batch": batch, "hidden": wl.hidden, "mlp": wl.mlp, "us_per_call": us,
+            "launches_per_call": 3, "w1_read_plus_dw1_write_bytes": nbytes,
+            "gbs": nbytes / (us / 1e6) / 1e9, "loss": float(loss.item())}
+
+
 def run_gate_point(args, dev, stream, prefill: int = 4096, steps: int = 256):
     """The gate-overhead point: the default workload's shapes with a short history."""
     w = oda_synth.scaled(oda_synth.WORKLOADS[args.workload], prefill=prefill,
@@ -701,6 +738,7 @@ def run_oda(args, dist: Dist):
 
     if w.name == DEFAULT_WORKLOAD:
         result["context_parallel_1gpu"] = cp_emulation(s, w, stream)
+        result["recall_train_grad"] = run_train_grad(w, dev, stream)
 
     # ---- end to end through the same API: host inputs in, selected output out ----
     if E2E:

@@ -89,8 +89,9 @@ typedef struct {
 } oda_kv;
 
 /* Bytes of workspace the decode calls need for `batch` sequences on the current device. The
- * workspace holds split partials and merge tickets; it must be zero-filled once before its
- * first use and is left zero-filled by every call, so one buffer serves any number of calls
+ * workspace holds split partials and merge tickets; the tickets must be zero before its
+ * first use (zero-fill the buffer once) and every call leaves them zero again, so one buffer
+ * serves any number of calls
  * issued in stream order. Returns ODA_OK or an error code. */
 int oda_decode_workspace_size(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads,
                               size_t* bytes);
@@ -241,8 +242,8 @@ int oda_gate_schedule(const float* u, int32_t batch, float rho, int32_t* gate_ou
  * (nullable u64[2]) is given, adds the number of gated sequences to full_count[0] and 1 to
  * full_count[1] when at least one sequence is gated; and, if graph_cond_handle != 0 (a
  * cudaGraphConditionalHandle), sets that graph condition to 1 iff any sequence is gated.
- * mlp must be a multiple of 64; hidden >= 1. ws: oda_recall_workspace_size() bytes, zeroed
- * once and left zeroed. */
+ * mlp must be a multiple of 64; hidden >= 1. ws: oda_recall_workspace_size() bytes, zero-
+ * filled once before first use; its tickets are left zero, its partials are scratch. */
 int oda_recall_workspace_size(int32_t batch, int32_t hidden, int32_t mlp, size_t* bytes);
 int oda_recall_score(const float* h_prev, const float* emb, const void* h_local,
                      int32_t h_local_dtype, int32_t batch, int32_t hidden, int32_t mlp,
@@ -250,6 +251,25 @@ int oda_recall_score(const float* h_prev, const float* emb, const void* h_local,
                      float* q_out, int32_t* gate_out, unsigned long long* full_count,
                      unsigned long long graph_cond_handle, void* ws, size_t ws_bytes,
                      void* stream);
+
+/* ---- recall-head training objective ([ODA] 핵심 기여 and 접근 방법: the head is trained,
+ *      backbone frozen, by Huber regression with delta = 1 of q_t on the signed-log target
+ *      y_t = sign(d_t) log(1 + |d_t|) of the cost-adjusted gain d_t = g_t - lambda,
+ *      g_t = log p^F_t(x_{t+1}) - log p^L_t(x_{t+1})) ---------------------------------------
+ * Inputs as oda_recall_score, plus gain (device fp32 [batch], g_t), lambda and delta > 0.
+ * Computes q (written to q_out when non-null), loss = mean over the batch of Huber(q - y)
+ * (fp32 scalar at loss_out) and its gradient with respect to the head's parameters:
+ * dw1 fp32 [3 * hidden][mlp], db1 / dw2 fp32 [mlp], db2 fp32 [1]; all outputs are fully
+ * overwritten. batch <= 1024; mlp a multiple of 64. ws: oda_recall_train_workspace_size()
+ * bytes, zero-filled once before first use (its ticket is left zero, the rest is scratch).
+ * Three kernel launches; deterministic. */
+int oda_recall_train_workspace_size(int32_t batch, int32_t hidden, int32_t mlp, size_t* bytes);
+int oda_recall_loss_grad(const float* h_prev, const float* emb, const void* h_local,
+                         int32_t h_local_dtype, int32_t batch, int32_t hidden, int32_t mlp,
+                         const float* w1, const float* b1, const float* w2, float b2,
+                         const float* gain, float lambda, float delta, float* q_out,
+                         float* loss_out, float* dw1, float* db1, float* dw2, float* db2,
+                         void* ws, size_t ws_bytes, void* stream);
 
 /* ---- Step runtime: one whole ODA decode step as one CUDA graph ([ODA] 개발자 관점: Local,
  *      the FP32 recall head and the conditional Full recompute in one GPU execution stream,

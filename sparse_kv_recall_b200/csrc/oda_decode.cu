@@ -30,8 +30,7 @@ constexpr int kStageBytes = 2 * kPageBytes;
 constexpr int kCtasPerSm = 2;
 constexpr int kMaxBatch = 1024;
 constexpr int kMaxGroup = 4;
-constexpr int kMinShare = 8;            // units per CTA at least: bounds merge fan-in
-constexpr int kMergeChunk = 32;         // partials staged in shared memory at a time
+constexpr int kMinShare = 4;            // units per CTA at least (one page per warp)
 
 static_assert(kThreads == kHeadDim, "merge maps one thread per output dim");
 
@@ -84,11 +83,39 @@ struct Vpl {
   static constexpr int value = G >= 2 ? G / 2 : 1;  // softmax values each lane owns
 };
 
-// One page: scores, online-softmax update, P.V accumulation.
+// Packed fp32 pairs: sm_100's fma.rn.f32x2 / mul.rn.f32x2 run two independent fp32 lanes per
+// instruction, each rounded exactly as fmaf / __fmul_rn would round it.
+typedef unsigned long long f2_t;
+
+__device__ __forceinline__ f2_t f2_pack(float lo, float hi) {
+  f2_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f2_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
+  f2_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2_t f2_mul(f2_t a, f2_t b) {
+  f2_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// A bf16 pair (low half = lower index) widened exactly to an fp32 pair.
+__device__ __forceinline__ f2_t bf16x2_widen(uint32_t w) {
+  return f2_pack(bf16lo(w), bf16hi(w));
+}
+
+// One page: scores, online-softmax update, P.V accumulation. q2[gg][j] holds the scaled
+// query dims (8 li + 2j, 8 li + 2j + 1) of head gg; acc[gg][j] the same dims of its P.V sum.
 template <int G>
-__device__ __forceinline__ void page_step(const unsigned char* stage, const float (&qf)[G][8],
+__device__ __forceinline__ void page_step(const unsigned char* stage, const f2_t (&q2)[G][4],
                                           float (&m_run)[Vpl<G>::value],
-                                          float (&l_run)[Vpl<G>::value], float (&acc)[G][8],
+                                          float (&l_run)[Vpl<G>::value], f2_t (&acc)[G][4],
                                           float* ps, const SeqPlan& sp, int lp, int lane,
                                           unsigned& rows_vis) {
   constexpr int VPL = Vpl<G>::value;
@@ -99,14 +126,18 @@ __device__ __forceinline__ void page_step(const unsigned char* stage, const floa
   float sc[8 * G];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    float kf[8];
-    unpack8(K[(2 * k + half) * 16 + li], kf);
+    const uint4 kw = K[(2 * k + half) * 16 + li];
+    const f2_t kp[4] = {bf16x2_widen(kw.x), bf16x2_widen(kw.y), bf16x2_widen(kw.z),
+                        bf16x2_widen(kw.w)};
 #pragma unroll
     for (int gg = 0; gg < G; ++gg) {
-      float s = 0.f;
+      // even and odd dims accumulate in the two lanes of a pair, then add
+      f2_t s2 = f2_mul(q2[gg][0], kp[0]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) s = fmaf(qf[gg][e], kf[e], s);
-      sc[k * G + gg] = s;
+      for (int j = 1; j < 4; ++j) s2 = f2_fma(q2[gg][j], kp[j], s2);
+      float lo, hi;
+      f2_unpack(s2, lo, hi);
+      sc[k * G + gg] = lo + hi;
     }
   }
   reduce_scatter<8 * G, 8>(sc, lane);
@@ -139,18 +170,21 @@ __device__ __forceinline__ void page_step(const unsigned char* stage, const floa
 #pragma unroll
   for (int gg = 0; gg < G; ++gg) {
     const float al = ashare[half * G + gg];
+    const f2_t al2 = f2_pack(al, al);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[gg][e] *= al;
+    for (int j = 0; j < 4; ++j) acc[gg][j] = f2_mul(acc[gg][j], al2);
   }
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    float vf[8];
-    unpack8(V[(2 * k + half) * 16 + li], vf);
+    const uint4 vw = V[(2 * k + half) * 16 + li];
+    const f2_t vp[4] = {bf16x2_widen(vw.x), bf16x2_widen(vw.y), bf16x2_widen(vw.z),
+                        bf16x2_widen(vw.w)};
 #pragma unroll
     for (int gg = 0; gg < G; ++gg) {
       const float pk = pshare[(half * 8 + k) * G + gg];
+      const f2_t pp = f2_pack(pk, pk);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[gg][e] = fmaf(pk, vf[e], acc[gg][e]);
+      for (int j = 0; j < 4; ++j) acc[gg][j] = f2_fma(pp, vp[j], acc[gg][j]);
     }
   }
   __syncwarp();
@@ -274,8 +308,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   int Pe = (int)min((long long)P, (T + kMinShare - 1) / kMinShare);
   // When every non-empty sequence has the same page count, a multiple of (non-empty
   // sequences x Hkv) CTAs makes every share fall inside one (b, g), so no CTA has to finish
-  // one piece before it can start streaming the next.
-  if (s_align > 0 && Pe >= s_align) Pe -= Pe % s_align;
+  // one piece before it can start streaming the next. Rounding up (when the grid has the
+  // CTAs) rather than down keeps the largest share at ceil(T / Pe) <= kMinShare units, i.e.
+  // at most one page per warp, so no warp of a short launch holds up its (b, g)'s merge.
+  // Rounding up never exceeds T: T = s_align x (pages per sequence).
+  if (s_align > 0) {
+    const int up = (Pe + s_align - 1) / s_align * s_align;
+    if (up <= P) Pe = up;
+    else if (Pe >= s_align) Pe -= Pe % s_align;
+  }
   long long x = c < Pe ? (T * c) / Pe : 0;
   const long long x_end = c < Pe ? (T * (c + 1)) / Pe : 0;
   while (x < x_end) {
@@ -298,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     const size_t head_off = (size_t)g * (kPage * kHeadDim);
     const size_t page_stride = (size_t)Hkv * kPage * kHeadDim;
 
-    float m_run[VPL], l_run[VPL], acc[G][8];
+    float m_run[VPL], l_run[VPL];
+    f2_t acc[G][4];
 #pragma unroll
     for (int u = 0; u < VPL; ++u) {
       m_run[u] = -INFINITY;
@@ -307,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
 #pragma unroll
     for (int gg = 0; gg < G; ++gg)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[gg][e] = 0.f;
+      for (int j = 0; j < 4; ++j) acc[gg][j] = f2_pack(0.f, 0.f);
 
     const int first = j0 + warp;
     const int cnt = first < j1 ? (j1 - first + kWarps - 1) / kWarps : 0;
@@ -334,14 +376,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     __syncwarp();
     dep_wait();
 
-    float qf[G][8];
+    f2_t q2[G][4];
 #pragma unroll
     for (int gg = 0; gg < G; ++gg) {
       const uint4 qv = *reinterpret_cast<const uint4*>(
           p.q + ((size_t)b * p.hq + g * G + gg) * kHeadDim + 8 * li);
-      unpack8(qv, qf[gg]);
+      float qf[8];
+      unpack8(qv, qf);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) qf[gg][e] *= p.scale_log2;
+      for (int j = 0; j < 4; ++j)
+        q2[gg][j] = f2_pack(qf[2 * j] * p.scale_log2, qf[2 * j + 1] * p.scale_log2);
     }
 
     for (int n = 0; n < cnt && !dead; ++n) {
@@ -373,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
           fence_proxy_async_smem();  // this stage is refilled by a bulk copy later
           __syncwarp();
         }
-        page_step<G>(st, qf, m_run, l_run, acc, ps, sp, r.lp, lane, rows_vis);
+        page_step<G>(st, q2, m_run, l_run, acc, ps, sp, r.lp, lane, rows_vis);
         ++pages_read;
       }
       __syncwarp();
@@ -392,7 +436,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       v += __shfl_xor_sync(0xffffffffu, v, 2);
       lsum[u] = v;
     }
+    if (p.stats != nullptr && lane == 0 && (rows_vis | pages_read)) {
+      atomicAdd(&s_rows, (unsigned long long)rows_vis);
+      atomicAdd(&s_pages, (unsigned long long)pages_read);
+    }
+    rows_vis = 0;
+    pages_read = 0;
     __syncthreads();  // every warp is done with its stages: reuse them as merge scratch
+    if (p.stats != nullptr && tid == 0) {
+      // issued now, so that the counter updates complete while the merge runs
+      if (s_rows) atomicAdd(&p.stats[ODA_STAT_ROWS], s_rows);
+      if (s_pages) atomicAdd(&p.stats[ODA_STAT_PAGES], s_pages);
+      s_rows = 0;
+      s_pages = 0;
+    }
     float* Mw = reinterpret_cast<float*>(stages);  // [2 * kWarps][G]
     float* Lw = Mw + 2 * kWarps * G;               // [2 * kWarps][G]
     float* Aw = Lw + 2 * kWarps * G;               // [2 * kWarps][G][128]
@@ -408,8 +465,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
 #pragma unroll
     for (int gg = 0; gg < G; ++gg) {
       float4* dst = reinterpret_cast<float4*>(Aw + (sidx * G + gg) * kHeadDim + 8 * li);
-      dst[0] = make_float4(acc[gg][0], acc[gg][1], acc[gg][2], acc[gg][3]);
-      dst[1] = make_float4(acc[gg][4], acc[gg][5], acc[gg][6], acc[gg][7]);
+      float a[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) f2_unpack(acc[gg][j], a[2 * j], a[2 * j + 1]);
+      dst[0] = make_float4(a[0], a[1], a[2], a[3]);
+      dst[1] = make_float4(a[4], a[5], a[6], a[7]);
     }
     __syncthreads();
     float o[G], l2[G];
@@ -452,12 +512,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       if (s_last) {
         // Merge the n_contrib partials in fixed order: log-sums into shared memory (stage
         // memory is free again), per-head max and weights by one warp per head, then every
-        // thread sums its dim over the partials with independent loads in flight.
+        // thread sums its dim over the partials with independent loads in flight. Partials
+        // are staged through shared memory, as many at a time as the stage memory holds
+        // (every one of a short launch's partials at once), by 16-byte asynchronous copies
+        // all in flight together; the first chunk is requested along with the log-sums, so
+        // one L2 round trip brings both.
         const size_t s0 = (size_t)c_first + bg;
         float* sw = reinterpret_cast<float*>(stages);  // [n_contrib][G] log-sums -> weights
         float* sml = sw + n_contrib * G;                // [G] max, [G] weight sum
         float* so = sml + 2 * G + (4 - (n_contrib * G + 2 * G) % 4) % 4;  // float4-aligned
+        const int chunk = (int)((kWarps * kStages * kStageBytes -
+                                 (size_t)(so - sw) * sizeof(float)) / (G * kHeadDim * sizeof(float)));
+        const float4* src = reinterpret_cast<const float4*>(p.ws_o + s0 * G * kHeadDim);
+        float4* dst4 = reinterpret_cast<float4*>(so);
+        auto stage_chunk = [&](int s_lo) {  // issue only; cp_async_wait_all completes it
+          const int n4 = min(chunk, n_contrib - s_lo) * G * kHeadDim / 4;
+          const float4* src_c = src + (size_t)s_lo * G * kHeadDim / 4;
+          for (int i = tid; i < n4; i += kThreads) cp_async16(dst4 + i, src_c + i);
+        };
+        stage_chunk(0);
         for (int i = tid; i < n_contrib * G; i += kThreads) sw[i] = __ldcg(&p.ws_lse[s0 * G + i]);
+        cp_async_wait_all();
         __syncthreads();
         if (warp < G) {
           float m = -INFINITY;
@@ -478,21 +553,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
             sml[G + warp] = sum;
           }
         }
+        __syncthreads();  // weights and the first chunk are in shared memory
         float a[G];
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) a[gg] = 0.f;
-        // Partials are staged through shared memory kMergeChunk at a time with independent
-        // 16-byte loads, then summed in fixed order by the thread that owns each dim.
-        const float4* src = reinterpret_cast<const float4*>(p.ws_o + s0 * G * kHeadDim);
-        float4* dst4 = reinterpret_cast<float4*>(so);
-        for (int s_lo = 0; s_lo < n_contrib; s_lo += kMergeChunk) {
-          const int ns = min(kMergeChunk, n_contrib - s_lo);
-          const int n4 = ns * G * kHeadDim / 4;
-          const float4* src_c = src + (size_t)s_lo * G * kHeadDim / 4;
-          __syncthreads();
-#pragma unroll 8
-          for (int i = tid; i < n4; i += kThreads) dst4[i] = __ldcg(src_c + i);
-          __syncthreads();
+        for (int s_lo = 0; s_lo < n_contrib; s_lo += chunk) {
+          const int ns = min(chunk, n_contrib - s_lo);
+          if (s_lo > 0) {
+            __syncthreads();  // everyone is done with the previous chunk
+            stage_chunk(s_lo);
+            cp_async_wait_all();
+            __syncthreads();
+          }
           for (int s = 0; s < ns; ++s)
 #pragma unroll
             for (int gg = 0; gg < G; ++gg)
@@ -530,18 +602,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
         l2[gg] = -INFINITY;
       }
       write_final<G>(p, b, bg % Hkv, o, l2);
-    }
-  }
-
-  if (p.stats != nullptr) {
-    if (lane == 0) {
-      atomicAdd(&s_rows, (unsigned long long)rows_vis);
-      atomicAdd(&s_pages, (unsigned long long)pages_read);
-    }
-    __syncthreads();
-    if (tid == 0) {
-      if (s_rows) atomicAdd(&p.stats[ODA_STAT_ROWS], s_rows);
-      if (s_pages) atomicAdd(&p.stats[ODA_STAT_PAGES], s_pages);
     }
   }
 }

@@ -15,16 +15,9 @@
 
 #include "oda_common.cuh"
 #include "oda_internal.h"
+#include "oda_recall.cuh"
 
 namespace oda {
-
-constexpr int kRThreads = 256;
-constexpr int kColTile = 64;
-constexpr int kRowGroups = kRThreads / kColTile;  // 4
-constexpr int kRows = 256;                        // rows of W1 per CTA
-constexpr int kRowsPerThread = kRows / kRowGroups;
-constexpr int kBTile = 8;                         // sequences per pass over the slab
-constexpr int kSlabChunk = 16;                    // slab partials in flight per thread
 
 struct RecallWs {
   size_t z_off, q_off, ticket_off, total;
@@ -44,15 +37,8 @@ static RecallWs recall_ws(int batch, int hidden, int mlp) {
   return w;
 }
 
-__device__ __forceinline__ float gelu_erf(float z) {
-  return 0.5f * z * (1.f + erff(z * 0.70710678118654752f));
-}
-
 struct RecallParams {
-  const float* h_prev;
-  const float* emb;
-  const void* h_local;
-  int h_local_bf16;
+  RecallInputs in;
   int batch, hidden, mlp;
   const float* w1;
   const float* b1;
@@ -67,16 +53,6 @@ struct RecallParams {
   float* q_part;      // [tiles][batch]
   unsigned* tickets;  // [tiles + 1]
 };
-
-__device__ __forceinline__ float x_at(const RecallParams& p, int b, int r) {
-  const int H = p.hidden;
-  if (r < H) return p.h_prev[(size_t)b * H + r];
-  if (r < 2 * H) return p.emb[(size_t)b * H + r - H];
-  const size_t i = (size_t)b * H + (r - 2 * H);
-  if (p.h_local_bf16)
-    return __bfloat162float(static_cast<const __nv_bfloat16*>(p.h_local)[i]);
-  return static_cast<const float*>(p.h_local)[i];
-}
 
 __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p) {
   __shared__ float xs[kBTile][kRows];
@@ -94,44 +70,14 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
   const int gcol = tile * kColTile + col;
 
   float wv[kRowsPerThread];  // this thread's W1 column over its rows, all loads in flight
-#pragma unroll
-  for (int i = 0; i < kRowsPerThread; ++i) {
-    const int r = rg + i * kRowGroups;
-    wv[i] = r < nrows ? __ldg(&p.w1[(size_t)(r0 + r) * p.mlp + gcol]) : 0.f;
-  }
+  load_w1_slab(p.w1, p.mlp, r0, nrows, gcol, rg, wv);
   // W1 is constant, so its loads above may overlap the previous kernel (the last Local
   // layer, which writes h_local); slabs that read h_local rows wait for it only now.
   if (r0 + nrows > 2 * p.hidden) griddep_wait();
   griddep_launch_dependents();
 
   // ---- partial z of this slab for every sequence ----
-  for (int b0 = 0; b0 < p.batch; b0 += kBTile) {
-    const int nb = min(kBTile, p.batch - b0);
-    for (int i = tid; i < kBTile * kRows; i += kRThreads) {
-      const int bb = i / kRows, r = i % kRows;
-      xs[bb][r] = (bb < nb && r < nrows) ? x_at(p, b0 + bb, r0 + r) : 0.f;
-    }
-    __syncthreads();
-    float acc[kBTile];
-#pragma unroll
-    for (int bb = 0; bb < kBTile; ++bb) acc[bb] = 0.f;
-#pragma unroll
-    for (int i = 0; i < kRowsPerThread; ++i) {
-      const int r = rg + i * kRowGroups;
-#pragma unroll
-      for (int bb = 0; bb < kBTile; ++bb) acc[bb] = fmaf(xs[bb][r], wv[i], acc[bb]);
-    }
-#pragma unroll
-    for (int bb = 0; bb < kBTile; ++bb) red[rg][bb][col] = acc[bb];
-    __syncthreads();
-    if (rg == 0) {
-      for (int bb = 0; bb < nb; ++bb) {
-        const float z = red[0][bb][col] + red[1][bb][col] + red[2][bb][col] + red[3][bb][col];
-        p.z_part[((size_t)slab * p.batch + b0 + bb) * p.mlp + gcol] = z;
-      }
-    }
-    __syncthreads();
-  }
+  slab_partial_z(p.in, wv, p.batch, p.mlp, slab, r0, nrows, gcol, xs, red, p.z_part);
 
   // ---- last slab of this column tile: z, GELU, w2 (summed over the tile's columns) ----
   __threadfence();
@@ -147,17 +93,7 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
     const int b = b0 + bl;
     float v = 0.f;
     if (b < p.batch) {
-      const float* zp = p.z_part + (size_t)b * p.mlp + gcol;
-      const size_t sstride = (size_t)p.batch * p.mlp;
-      float z = 0.f;
-      for (int s0 = 0; s0 < slabs; s0 += kSlabChunk) {
-        float part[kSlabChunk];
-#pragma unroll
-        for (int u = 0; u < kSlabChunk; ++u)
-          part[u] = (s0 + u < slabs) ? __ldcg(zp + (size_t)(s0 + u) * sstride) : 0.f;
-#pragma unroll
-        for (int u = 0; u < kSlabChunk; ++u) z += part[u];
-      }
+      const float z = sum_slabs(p.z_part, b, gcol, p.batch, p.mlp, slabs);
       v = gelu_erf(z + p.b1[gcol]) * p.w2[gcol];
     }
 #pragma unroll
@@ -217,10 +153,11 @@ int launch_recall(const float* h_prev, const float* emb, const void* h_local, in
   const RecallWs wl = recall_ws(batch, hidden, mlp);
   if (ws_bytes < wl.total) return ODA_ERR_WORKSPACE_TOO_SMALL;
   RecallParams p;
-  p.h_prev = h_prev;
-  p.emb = emb;
-  p.h_local = h_local;
-  p.h_local_bf16 = h_local_dtype == ODA_BF16;
+  p.in.h_prev = h_prev;
+  p.in.emb = emb;
+  p.in.h_local = h_local;
+  p.in.h_local_bf16 = h_local_dtype == ODA_BF16;
+  p.in.hidden = hidden;
   p.batch = batch;
   p.hidden = hidden;
   p.mlp = mlp;

@@ -124,6 +124,9 @@ _SIGNATURES = {
     "oda_visible_mask_ex": (ctypes.c_int, [_KV, _VIS, _P, _I, _P]),
     "oda_merge_partials": (ctypes.c_int, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _P]),
     "oda_gate_schedule": (ctypes.c_int, [_P, _I, _F, _P, _P, ctypes.c_ulonglong, _P]),
+    "oda_recall_train_workspace_size": (ctypes.c_int, [_I, _I, _I, ctypes.POINTER(_SZ)]),
+    "oda_recall_loss_grad": (ctypes.c_int, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _F, _P, _F,
+                                            _F, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "oda_recall_score": (ctypes.c_int, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _F, _F, _P, _P, _P,
                                         ctypes.c_ulonglong, _P, _SZ, _P]),
     "oda_step_graph_create": (ctypes.c_int, [ctypes.POINTER(oda_step_desc), _P,
@@ -433,3 +436,28 @@ class StepGraph:
             self.close()
         except Exception:
             pass
+
+
+def oda_recall_train_workspace_size(batch: int, hidden: int, mlp: int) -> int:
+    n = _SZ(0)
+    _check(load().oda_recall_train_workspace_size(batch, hidden, mlp, ctypes.byref(n)),
+           "oda_recall_train_workspace_size")
+    return n.value
+
+
+def oda_recall_loss_grad(h_prev, emb, h_local, w1, b1, w2, b2: float, gain, lam: float, ws,
+                         loss, dw1, db1, dw2, db2, delta: float = 1.0, q_out=None, stream=None):
+    """Mean Huber loss of the recall head on the signed-log targets of `gain` (fp32 [B]) and
+    its gradient; loss / db2 are fp32 [1] device tensors, dw1 / db1 / dw2 shaped like the
+    weights."""
+    batch, hidden = h_prev.shape
+    _check(load().oda_recall_loss_grad(
+        _ptr(h_prev, torch.float32, "h_prev"), _ptr(emb, torch.float32, "emb"),
+        _ptr(h_local, None, "h_local"), _out_dtype(h_local), batch, hidden, w1.shape[1],
+        _ptr(w1, torch.float32, "w1"), _ptr(b1, torch.float32, "b1"), _ptr(w2, torch.float32, "w2"),
+        float(b2), _ptr(gain, torch.float32, "gain"), float(lam), float(delta),
+        _ptr(q_out, torch.float32, "q_out"), _ptr(loss, torch.float32, "loss"),
+        _ptr(dw1, torch.float32, "dw1"), _ptr(db1, torch.float32, "db1"),
+        _ptr(dw2, torch.float32, "dw2"), _ptr(db2, torch.float32, "db2"),
+        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+        "oda_recall_loss_grad")

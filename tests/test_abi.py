@@ -158,3 +158,25 @@ def test_merge_and_schedule_argument_checks(lib):
     assert lib.oda_gate_schedule(0x1000, 4, float("nan"), 0x2000, None, 0, None) == I
     assert lib.oda_gate_schedule(None, 4, 0.5, 0x2000, None, 0, None) == I
     assert lib.oda_gate_schedule(0x1000, 0, 0.5, 0x2000, None, 0, None) == OK
+
+
+def test_recall_training_argument_checks(lib):
+    I = oda.ODA_ERR_INVALID_ARG
+    n = ctypes.c_size_t(0)
+    assert lib.oda_recall_train_workspace_size(1025, 2048, 256, ctypes.byref(n)) == I
+    assert lib.oda_recall_train_workspace_size(8, 2048, 100, ctypes.byref(n)) == I
+    assert lib.oda_recall_train_workspace_size(8, 2048, 256, ctypes.byref(n)) == oda.ODA_OK
+    need = n.value
+    assert need > 0
+
+    def call(batch=8, mlp=256, delta=1.0, gain=0xa, ws_bytes=None):
+        return lib.oda_recall_loss_grad(0x1, 0x2, 0x3, 0, batch, 2048, mlp, 0x4, 0x5, 0x6, 0.0,
+                                        gain, 0.0, delta, None, 0xb, 0xc, 0xd, 0xe, 0xf, 0x10,
+                                        need if ws_bytes is None else ws_bytes, None)
+    assert call(delta=0.0) == I
+    assert call(delta=float("inf")) == I
+    assert call(gain=None) == I
+    assert call(mlp=96) == I
+    assert call(batch=2000) == I
+    assert call(ws_bytes=16) == oda.ODA_ERR_WORKSPACE_TOO_SMALL
+    assert call(batch=0) == oda.ODA_OK
