@@ -212,7 +212,10 @@ class Setup:
         self.w = oda_synth.scaled(w, seed=w.seed + 1000 * seed_offset)
         w = self.w
         self.lengths = oda_synth.prefill_lengths(w)
-        self.layout = oda_synth.make_layout(w, extra_tokens=n_steps_total + 4, device=dev)
+        # a fixed capacity keeps the page layout, hence the synthetic cache, the same whatever
+        # number of steps a run takes
+        self.layout = oda_synth.make_layout(w, extra_tokens=max(n_steps_total + 4, 8192),
+                                            device=dev)
         self.caches = [oda_synth.make_kv_cache(w, self.layout, l, device=dev) for l in range(w.layers)]
         rw = oda_synth.make_recall_weights(w, device=dev)
         self.recall = (rw.w1, rw.b1, rw.w2, rw.b2)
@@ -238,16 +241,23 @@ def launches_per_step(w, phases: int, steps: int, conditional: bool = True) -> i
 
 
 def calibrate_theta(s, w, C: int, step: int):
-    """theta = (1 - target rho) quantile of q over C Local-only steps (graphs captured with
-    theta = +inf); returns (theta, next step index)."""
-    qs = []
-    for _ in range(C):
-        s.feed(step)
-        s.eng.launch(step)
-        qs.append(s.eng.q_out.clone())
-        step += 1
-    q = torch.cat(qs).double().cpu().numpy()
-    return float(np.quantile(q, 1.0 - w.target_rho)), step
+    """theta for the target Full-call rate, in two passes: the (1 - target rho) quantile of q
+    over C/2 Local-only steps (graphs captured with theta = +inf), then the same quantile
+    over C/2 steps gated at that first theta (q then sees the h_{t-1} trajectory that gating
+    produces); returns (theta, next step index)."""
+    def collect(n):
+        nonlocal step
+        qs = []
+        for _ in range(n):
+            s.feed(step)
+            s.eng.launch(step)
+            qs.append(s.eng.q_out.clone())
+            step += 1
+        return torch.cat(qs).double().cpu().numpy()
+    theta = float(np.quantile(collect(C // 2), 1.0 - w.target_rho))
+    s.eng.set_theta(theta)
+    theta = float(np.quantile(collect(C - C // 2), 1.0 - w.target_rho))
+    return theta, step
 
 
 def phase_breakdown(s, w, theta: float, PH: int, step: int, stream):
@@ -262,14 +272,22 @@ def phase_breakdown(s, w, theta: float, PH: int, step: int, stream):
             e.record(stream)
     torch.cuda.synchronize()
     gated = []
+    gates = torch.zeros((PH, w.batch), dtype=torch.int32, device=eng.gate.device)
+    first = step
     for i in range(PH):
         before = eng.full_count[1].clone()
         eng.set_events(step, evs[i])
         s.feed(step)
         eng.launch(step)
+        gates[i].copy_(eng.gate, non_blocking=True)
         gated.append(before)
         step += 1
     torch.cuda.synchronize()
+    # Full-phase bytes of each step: its gated sequences' whole histories at every layer
+    lens = np.array(s.lengths, dtype=np.float64)
+    g_h = gates.cpu().numpy().astype(np.float64)
+    full_bytes = [float((g_h[i] * (lens + first + i + 1)).sum()) * w.num_kv_heads * ROW_BYTES
+                  * w.layers for i in range(PH)]
     counts = torch.stack(gated).cpu().tolist() + [int(eng.full_count[1].item())]
     ran_full = [counts[i + 1] > counts[i] for i in range(PH)]
     t_local = [evs[i][0].elapsed_time(evs[i][1]) for i in range(PH)]
@@ -282,8 +300,6 @@ def phase_breakdown(s, w, theta: float, PH: int, step: int, stream):
     T_step, T_loc = mean(t_step), mean(t_local)
     T_full_exec = sum(t_full[i] for i in full_steps) / PH if PH else 0.0
     gate_over = (T_step - T_loc - T_full_exec) / T_step if T_step else None
-    ctx = np.mean(s.lengths) + step - PH / 2
-    full_launch_bytes = w.batch * (ctx + 1) * w.num_kv_heads * ROW_BYTES
     local_rows = sum(min(n + step - PH / 2 + 1, w.sink + w.window) for n in s.lengths)
     eng.timing = False
     eng.set_theta(theta)
@@ -296,8 +312,9 @@ def phase_breakdown(s, w, theta: float, PH: int, step: int, stream):
                              "node timed without PDL between event nodes",
         "local_phase_kv_gbs": (w.layers * w.num_kv_heads * local_rows * ROW_BYTES
                                / (T_loc / 1e3) / 1e9) if T_loc else None,
-        "full_phase_kv_gbs": (w.layers * full_launch_bytes / (mean([t_full[i] for i in full_steps]) / 1e3)
-                              / 1e9) if full_steps else None,
+        "full_phase_kv_gbs": (sum(full_bytes[i] for i in full_steps)
+                              / (sum(t_full[i] for i in full_steps) / 1e3) / 1e9)
+                             if full_steps else None,
     }, step
 
 
@@ -315,38 +332,58 @@ def timed_steps(s, n: int, step: int, stream):
     return a.elapsed_time(b) / n, step
 
 
-def gate_cost(s, w, theta: float, n: int, step: int, stream):
+def gate_cost(s, w, theta: float, n: int, step: int, stream, rounds: int = 4):
     """Step time of the same PDL-chained graphs (no event nodes inside) at the calibrated
     theta, at theta = +inf (Local + recall + skipped IF node), at theta = -inf (every step
-    runs Full) and as a Local-only graph; the recall head and the IF machinery cost
-    T(+inf) - T(Local only), the Full phase T(-inf) - T(+inf)."""
+    runs Full), as a Local-only graph and as a Local + recall graph (no IF node); the recall
+    head and the IF machinery cost T(+inf) - T(Local only), split into the recall head
+    T(Local + recall) - T(Local only) and the skipped IF node T(+inf) - T(Local + recall);
+    the Full phase costs T(-inf) - T(+inf). The variants are captured once and timed in
+    `rounds` interleaved rounds of n steps each; each figure is the median over rounds."""
     from sparse_kv_recall_b200 import oda
     eng = s.eng
-    out = {}
-    fc0 = eng.full_count.clone()
-    for name, th, phases in [("oda", theta, 0), ("theta_plus_inf", math.inf, 0),
-                             ("theta_minus_inf", -math.inf, 0),
-                             ("local_only", math.inf, oda.ODA_PHASE_LOCAL)]:
-        eng.phases = phases
-        eng.set_theta(th)
-        _, step = timed_steps(s, 8, step, stream)            # settle after re-capture
-        if name == "oda":
+    variants = [("oda", theta, 0), ("theta_plus_inf", math.inf, 0),
+                ("theta_minus_inf", -math.inf, 0), ("local_only", math.inf, oda.ODA_PHASE_LOCAL),
+                ("local_recall", math.inf, oda.ODA_PHASE_LOCAL | oda.ODA_PHASE_RECALL)]
+    graphs = {name: eng.capture(th, ph) for name, th, ph in variants}
+    times = {name: [] for name, _, _ in variants}
+    gated = 0
+    for _ in range(rounds):
+        for name, _, _ in variants:
+            g = graphs[name]
+            for _ in range(4):                                # settle on this graph
+                s.feed(step)
+                g[step % 2].launch()
+                step += 1
             fc0 = eng.full_count.clone()
-        out[name], step = timed_steps(s, n, step, stream)
-        if name == "oda":
-            out["rho_realised"] = float((eng.full_count - fc0)[0].item()) / (w.batch * n)
-    eng.phases = 0
-    eng.set_theta(theta)
-    T = out
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n):
+                s.feed(step)
+                g[step % 2].launch()
+                step += 1
+            b.record(stream)
+            torch.cuda.synchronize()
+            times[name].append(a.elapsed_time(b) / n)
+            if name == "oda":
+                gated += int((eng.full_count - fc0)[0].item())
+    for g in graphs.values():
+        for x in g:
+            x.close()
+    T = {name: float(np.median(v)) for name, v in times.items()}
     overhead = T["theta_plus_inf"] - T["local_only"]
-    return {"ms_per_step": {k: v for k, v in T.items() if k.startswith(("oda", "theta", "local"))},
-            "rho_realised": T["rho_realised"],
+    return {"ms_per_step": T, "rounds": rounds, "steps_per_round": n,
+            "rho_realised": gated / float(w.batch * n * rounds),
             "ms_recall_and_if_node": overhead,
+            "ms_recall_head": T["local_recall"] - T["local_only"],
+            "ms_if_node_skipped": T["theta_plus_inf"] - T["local_recall"],
             "ms_full_phase": T["theta_minus_inf"] - T["theta_plus_inf"],
             "gate_overhead": overhead / T["oda"],
             "gate_overhead_def": "(T(theta=+inf) - T(Local-only graph)) / T(calibrated theta): "
                                  "recall head + IF node per step over the whole step, same "
-                                 "PDL-chained graphs, no event nodes inside"}, step
+                                 "PDL-chained graphs, no event nodes inside, medians of "
+                                 "interleaved rounds"}, step
 
 
 def step_variants(s, w, theta: float, rho: float, n: int, step: int, stream):
@@ -467,14 +504,14 @@ def run_gate_point(args, dev, stream, prefill: int = 4096, steps: int = 256):
     w = oda_synth.scaled(oda_synth.WORKLOADS[args.workload], prefill=prefill,
                          name=args.workload + "@%d" % prefill)
     C, W = 256, 8
-    s = Setup(w, 0, C + W + 5 * steps + 64, float("inf"), dev)
+    s = Setup(w, 0, C + W + 5 * 4 * (steps // 4 + 4) + steps + 64, float("inf"), dev)
     theta, step = calibrate_theta(s, w, C, 0)
     s.eng.set_theta(theta)
     for _ in range(W):
         s.feed(step)
         s.eng.launch(step)
         step += 1
-    res, step = gate_cost(s, w, theta, steps, step, stream)
+    res, step = gate_cost(s, w, theta, steps // 4, step, stream)
     ph, step = phase_breakdown(s, w, theta, steps, step, stream)
     assert int(s.eng.status.item()) == 0
     s.eng.close()
@@ -635,7 +672,7 @@ def run_oda(args, dist: Dist):
     GC = 0 if args.quick else 64
     E2E = 0 if (args.quick or args.no_e2e) else min(K, 256)
     VAR = 0 if args.quick else 128
-    total = C + W + K + PH + (4 * GC + 32 if GC else 0) + E2E + (2 * VAR + 16 if VAR else 0)
+    total = C + W + K + PH + (5 * 4 * (GC + 4) if GC else 0) + E2E + (2 * VAR + 16 if VAR else 0)
     s = Setup(w, dist.rank, total, float("inf") if w.theta is None else w.theta, dev,
               use_conditional=not args.no_conditional)
     eng = s.eng
@@ -728,13 +765,24 @@ def run_oda(args, dist: Dist):
     dur = float(np.mean([a.elapsed_time(b) for a, b in kevs]))
     ctx_tokens = int(eng.seq_lens.sum().item())
     alg = ctx_tokens * w.num_kv_heads * ROW_BYTES
-    achieved = alg / (dur / 1e3) / 1e9
+    achieved_alone = alg / (dur / 1e3) / 1e9
     traffic = profiled_traffic(ctx_tokens)
+    # The dominant kernel as the step runs it: the Full phase (w.layers launches chained with
+    # programmatic dependent launch) timed by event nodes at its boundaries, per launch; its
+    # bytes per launch at that phase's context. Alone: one launch between two events.
+    ph = result["phases"]
+    if ph.get("full_phase_kv_gbs"):
+        achieved, how = ph["full_phase_kv_gbs"], ("Full phase inside the step graph (%d launches "
+                                                  "between event nodes, PDL-chained)" % w.layers)
+        ms_launch = ph["ms_full_phase_when_run"] / w.layers
+    else:
+        achieved, how, ms_launch = achieved_alone, "one launch between two events", dur
     result["roofline"] = {"kernel": "oda_decode_full (decode_kernel<%d>)" % w.group,
                           "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                           "frac": achieved / peak, "traffic": traffic,
-                          "algorithmic_bytes": alg, "ms_per_launch": dur,
-                          "peak_kind": peak_kind + " (burst copy; kernel timed alone)"}
+                          "algorithmic_bytes": alg, "ms_per_launch": ms_launch, "timed": how,
+                          "achieved_alone": achieved_alone, "frac_alone": achieved_alone / peak,
+                          "ms_per_launch_alone": dur, "peak_kind": peak_kind + " (copy)"}
 
     if w.name == DEFAULT_WORKLOAD:
         result["context_parallel_1gpu"] = cp_emulation(s, w, stream)

@@ -114,6 +114,14 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
+// Arrive on a merge ticket: gpu-scope acquire-release add by one thread, after a CTA
+// barrier, publishes the CTA's partial and, for the last arrival, acquires all others.
+__device__ __forceinline__ unsigned ticket_arrive(unsigned* t) {
+  unsigned prev;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(t) : "memory");
+  return prev;
+}
+
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));

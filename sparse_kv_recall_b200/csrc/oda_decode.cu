@@ -211,14 +211,6 @@ __device__ __forceinline__ void write_final(const DecodeParams& p, int b, int g,
   }
 }
 
-// Arrive on a merge ticket: gpu-scope acquire-release add by one thread, after a CTA
-// barrier, publishes the CTA's partial and, for the last arrival, acquires all others.
-__device__ __forceinline__ unsigned ticket_arrive(unsigned* t) {
-  unsigned prev;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(t) : "memory");
-  return prev;
-}
-
 // CTA whose share contains flattened unit x (shares are [c*T/P, (c+1)*T/P), P <= T).
 __device__ __forceinline__ int cta_of(long long x, long long T, int P) {
   return (int)(((x + 1) * P - 1) / T);

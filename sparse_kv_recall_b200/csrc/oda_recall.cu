@@ -8,9 +8,10 @@
 // each, so the whole GPU streams W1 once per call for every sequence of the batch; each
 // thread holds its 64 W1 values in registers, all loads in flight at once. Per column tile,
 // the last slab CTA to finish (atomic ticket) sums the slabs' partial z in fixed order, one
-// (sequence, column) per thread with 16 loads in flight, and applies b1, GELU and w2; the
-// last column tile then forms q, the gate, the counters and the graph condition. Fixed
-// orders make every result bitwise reproducible.
+// (sequence, column) per thread with 24 loads in flight, and applies b1, GELU and w2; the
+// last column tile then forms q, the gate, the counters and the graph condition. For up to
+// four sequences one ticket over all CTAs replaces the two levels: the last CTA sums every
+// slab of every column itself. Fixed orders make every result bitwise reproducible.
 #include <math.h>
 
 #include "oda_common.cuh"
@@ -54,12 +55,33 @@ struct RecallParams {
   unsigned* tickets;  // [tiles + 1]
 };
 
-__global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p) {
+constexpr int kSmallBatch = 4;  // up to this many sequences: one ticket level (see below)
+
+// Gate, Full-call counters and the graph condition from this thread's q of sequence b.
+__device__ __forceinline__ void gate_one(const RecallParams& p, int b, float q,
+                                         unsigned* s_count) {
+  const int gate = q > p.theta ? 1 : 0;
+  p.q_out[b] = q;
+  p.gate_out[b] = gate;
+  if (gate) atomicAdd(s_count, 1u);
+}
+__device__ __forceinline__ void publish_gate(const RecallParams& p, unsigned count) {
+  if (p.full_count != nullptr && count) {
+    atomicAdd(&p.full_count[0], (unsigned long long)count);
+    atomicAdd(&p.full_count[1], 1ull);
+  }
+  if (p.use_cond) cudaGraphSetConditional(p.cond, count ? 1u : 0u);
+}
+
+// At most 104 registers: two Local CTAs and one recall CTA fit on an SM together, so the
+// recall head can start (programmatic dependent launch) while the last Local layer runs.
+__global__ void __maxnreg__(104) recall_kernel(const RecallParams p) {
   __shared__ float xs[kBTile][kRows];
   __shared__ float red[kRowGroups][kBTile][kColTile];
   __shared__ float qs[kRowGroups][2];
   __shared__ int s_last;
-  __shared__ unsigned s_any, s_count;
+  __shared__ unsigned s_count;
+  __shared__ float s_red[kRThreads / 32][kSmallBatch];
 
   const int tid = threadIdx.x;
   const int rg = tid / kColTile, col = tid % kColTile;
@@ -71,6 +93,9 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
 
   float wv[kRowsPerThread];  // this thread's W1 column over its rows, all loads in flight
   load_w1_slab(p.w1, p.mlp, r0, nrows, gcol, rg, wv);
+  // the final reduction's constants for column tid, in case this CTA ends up doing it
+  const float b1_own = tid < p.mlp ? __ldg(&p.b1[tid]) : 0.f;
+  const float w2_own = tid < p.mlp ? __ldg(&p.w2[tid]) : 0.f;
   // W1 is constant, so its loads above may overlap the previous kernel (the last Local
   // layer, which writes h_local); slabs that read h_local rows wait for it only now.
   if (r0 + nrows > 2 * p.hidden) griddep_wait();
@@ -79,13 +104,49 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
   // ---- partial z of this slab for every sequence ----
   slab_partial_z(p.in, wv, p.batch, p.mlp, slab, r0, nrows, gcol, xs, red, p.z_part);
 
+  // ---- small batches: one ticket over every CTA; the last one sums every slab of every
+  // column (all loads of a thread in flight together) and reduces q in the CTA, one global
+  // round trip shorter than the two-level reduction below ----
+  if (p.batch <= kSmallBatch) {
+    __syncthreads();  // the CTA's partials are written; thread 0 publishes them (release)
+    if (tid == 0) {
+      s_last = ticket_arrive(&p.tickets[tiles]) == (unsigned)(slabs * tiles - 1);
+      s_count = 0u;
+    }
+    __syncthreads();  // ... and the last CTA's thread 0 acquired everyone's partials
+    if (!s_last) return;
+#pragma unroll 1
+    for (int b = 0; b < p.batch; ++b) {
+      float v = 0.f;
+      for (int c = tid; c < p.mlp; c += kRThreads) {
+        const bool first = c == tid;  // this column's b1, w2 were fetched before the wait
+        v += gelu_erf(sum_slabs(p.z_part, b, c, p.batch, p.mlp, slabs) +
+                      (first ? b1_own : p.b1[c])) * (first ? w2_own : p.w2[c]);
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if ((tid & 31) == 0) s_red[tid >> 5][b] = v;
+    }
+    __syncthreads();
+    if (tid < p.batch) {
+      float q = 0.f;
+#pragma unroll
+      for (int w = 0; w < kRThreads / 32; ++w) q += s_red[w][tid];
+      gate_one(p, tid, q + p.b2, &s_count);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      publish_gate(p, s_count);
+      p.tickets[tiles] = 0u;
+    }
+    return;
+  }
+
   // ---- last slab of this column tile: z, GELU, w2 (summed over the tile's columns) ----
-  __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&p.tickets[tile], 1u) == (unsigned)(slabs - 1);
+  if (tid == 0) s_last = ticket_arrive(&p.tickets[tile]) == (unsigned)(slabs - 1);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   // Thread (bl, col) sums column gcol of sequence b0 + bl over every slab, kSlabChunk
   // independent loads in flight at a time, in fixed slab order.
   const int bl = tid / kColTile;
@@ -107,35 +168,21 @@ __global__ void __launch_bounds__(kRThreads) recall_kernel(const RecallParams p)
   if (tid == 0) p.tickets[tile] = 0u;
 
   // ---- last column tile: q, gate, counters, condition ----
-  __threadfence();
   __syncthreads();
   if (tid == 0) {
-    s_last = atomicAdd(&p.tickets[tiles], 1u) == (unsigned)(tiles - 1);
-    s_any = 0u;
+    s_last = ticket_arrive(&p.tickets[tiles]) == (unsigned)(tiles - 1);
     s_count = 0u;
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   for (int b = tid; b < p.batch; b += kRThreads) {
     float q = 0.f;
     for (int t = 0; t < tiles; ++t) q += __ldcg(&p.q_part[(size_t)t * p.batch + b]);
-    q += p.b2;
-    const int gate = q > p.theta ? 1 : 0;
-    p.q_out[b] = q;
-    p.gate_out[b] = gate;
-    if (gate) {
-      atomicAdd(&s_count, 1u);
-      s_any = 1u;
-    }
+    gate_one(p, b, q + p.b2, &s_count);
   }
   __syncthreads();
   if (tid == 0) {
-    if (p.full_count != nullptr && s_count) {
-      atomicAdd(&p.full_count[0], (unsigned long long)s_count);
-      atomicAdd(&p.full_count[1], 1ull);
-    }
-    if (p.use_cond) cudaGraphSetConditional(p.cond, s_any ? 1u : 0u);
+    publish_gate(p, s_count);
     p.tickets[tiles] = 0u;
   }
 }

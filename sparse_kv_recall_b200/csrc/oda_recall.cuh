@@ -16,7 +16,7 @@ constexpr int kRowGroups = kRThreads / kColTile;  // 4
 constexpr int kRows = 256;                        // rows of W1 per CTA
 constexpr int kRowsPerThread = kRows / kRowGroups;
 constexpr int kBTile = 8;                         // sequences per pass over the slab
-constexpr int kSlabChunk = 16;                    // slab partials in flight per thread
+constexpr int kSlabChunk = 24;                    // slab partials in flight per thread
 
 __device__ __forceinline__ float gelu_erf(float z) {
   return 0.5f * z * (1.f + erff(z * 0.70710678118654752f));
@@ -63,22 +63,22 @@ __device__ __forceinline__ void slab_partial_z(const RecallInputs& in,
   const int rg = tid / kColTile, col = tid % kColTile;
   for (int b0 = 0; b0 < batch; b0 += kBTile) {
     const int nb = min(kBTile, batch - b0);
-    for (int i = tid; i < kBTile * kRows; i += kRThreads) {
+    for (int i = tid; i < nb * kRows; i += kRThreads) {
       const int bb = i / kRows, r = i % kRows;
-      xs[bb][r] = (bb < nb && r < nrows) ? x_at(in, b0 + bb, r0 + r) : 0.f;
+      xs[bb][r] = r < nrows ? x_at(in, b0 + bb, r0 + r) : 0.f;
     }
     __syncthreads();
-    float acc[kBTile];
+    // only the nb sequences present (a batch of one does 1/8 of the FMAs of a full tile)
 #pragma unroll
-    for (int bb = 0; bb < kBTile; ++bb) acc[bb] = 0.f;
+    for (int bb = 0; bb < kBTile; ++bb) {
+      if (bb < nb) {
+        float acc = 0.f;
 #pragma unroll
-    for (int i = 0; i < kRowsPerThread; ++i) {
-      const int r = rg + i * kRowGroups;
-#pragma unroll
-      for (int bb = 0; bb < kBTile; ++bb) acc[bb] = fmaf(xs[bb][r], wv[i], acc[bb]);
+        for (int i = 0; i < kRowsPerThread; ++i)
+          acc = fmaf(xs[bb][rg + i * kRowGroups], wv[i], acc);
+        red[rg][bb][col] = acc;
+      }
     }
-#pragma unroll
-    for (int bb = 0; bb < kBTile; ++bb) red[rg][bb][col] = acc[bb];
     __syncthreads();
     if (rg == 0) {
       for (int bb = 0; bb < nb; ++bb) {

@@ -109,12 +109,10 @@ __global__ void __launch_bounds__(kRThreads) train_head_kernel(const TrainParams
     __syncthreads();
   }
   // the last column tile to finish forms q, the loss and dq
-  __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(p.ticket, 1u) == (unsigned)(tiles - 1);
+  if (tid == 0) s_last = ticket_arrive(p.ticket) == (unsigned)(tiles - 1);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   __shared__ float s_h[kMaxTrainBatch], s_dq[kMaxTrainBatch];
   const float inv_b = 1.f / (float)p.batch;
   for (int b = tid; b < p.batch; b += kRThreads) {

@@ -126,22 +126,29 @@ class OdaEngine:
         for g in self.graphs:
             g.close()
         self.theta = float(theta)
+        self.graphs = self.capture(self.theta, self.phases)
+
+    def capture(self, theta: float, phases: int = 0):
+        """An even/odd pair of step graphs over this engine's buffers with the given threshold
+        and phase mask, owned by the caller (launch graphs[step % 2]; close both when done).
+        The engine's own graphs are untouched."""
         v = self.v
         names = lambda p: [v["%s_%d" % (p, l)] for l in range(self.L)]
-        self.graphs = []
+        graphs = []
         for parity in (0, 1):
-            self.graphs.append(oda.StepGraph(
+            graphs.append(oda.StepGraph(
                 self.kvs, self.hq, self.sink, self.window, self.scale,
                 names("q_local"), names("k_local"), names("v_local"),
                 names("q_full"), names("k_full"), names("v_full"),
                 self._layer_out(parity), self.h[parity], v["emb"], self.w1, self.b1, self.w2,
-                self.b2, self.theta, self.q_out, self.gate, self.decode_ws, self.recall_ws,
+                self.b2, float(theta), self.q_out, self.gate, self.decode_ws, self.recall_ws,
                 full_count=self.full_count, lse=self.lse, local_layers=self.local_layers,
                 sinks=self.sinks, windows=self.windows,
                 gate_u=v["gate_u"] if self.random_rho is not None else None,
                 rho=self.random_rho or 0.0,
                 use_conditional=self.use_conditional, timing_events=self.timing,
-                phases=self.phases))
+                phases=phases))
+        return graphs
 
     def set_h_prev(self, h0: torch.Tensor, step: int = 0):
         """h_{t-1} that step `step` will read."""
