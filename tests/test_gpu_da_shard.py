@@ -129,6 +129,20 @@ def test_context_parallel_full_equals_full(parts):
     f, lf = c.out_buffers()
     _run(c, lambda: oda.oda_decode_full(c.kv, c.q, SCALE, f, c.ws, lse=lf))
     assert (out - f).abs().max().item() <= 2e-6 and (lse - lf).abs().max().item() <= 2e-5
+    # the exported plan of each shard is exactly its positions, and the shards tile 0..t
+    T = max(lens)
+    cover = np.zeros((c.B, T), dtype=np.int64)
+    for lo, hi in shards:
+        mask = torch.full((c.B, T), 7, dtype=torch.uint8, device="cuda")
+        _run(c, lambda: oda.oda_visible_mask_ex(c.kv, oda.shard_visibility(lo, hi), mask))
+        mk = mask.cpu().numpy()
+        for b, n in enumerate(lens):
+            want = np.zeros(T, dtype=np.uint8)
+            want[O.shard_positions(n - 1, lo, hi)] = 1
+            assert np.array_equal(mk[b], want)
+        cover += mk
+    assert all(np.array_equal(cover[b, :n], np.ones(n)) and not cover[b, n:].any()
+               for b, n in enumerate(lens))
 
 
 def test_context_parallel_commit_and_gate():

@@ -53,6 +53,33 @@ def test_local_matches_oracle(sink, window):
     assert c.stats[oda.ODA_STAT_ROWS].item() == 8 * rows
 
 
+def test_maximum_batch_local_and_full():
+    """The largest batch one launch takes (1024 sequences), ragged 1..700 tokens: every
+    sequence's attended-row count exactly, sampled sequences against the oracle."""
+    r = np.random.default_rng(11)
+    lens = [int(x) for x in r.integers(1, 701, size=1024)]
+    c = Case(lens, hq=16, hkv=8, seed=12, extra=0, spare_pages=0)
+    seqs = list(range(0, 1024, 41)) + [1023]
+    for name, fn, pos in [
+            ("local", lambda o, l: oda.oda_decode_local(c.kv, c.q, 4, 128, SCALE, o, c.ws, lse=l),
+             lambda b, t: O.local_positions(t, 4, 128)),
+            ("full", lambda o, l: oda.oda_decode_full(c.kv, c.q, SCALE, o, c.ws, lse=l),
+             lambda b, t: O.full_positions(t))]:
+        c.stats.zero_()
+        out, lse = c.out_buffers()
+        _run(c, lambda: fn(out, lse))
+        ref, rlse = c.oracle(pos, seqs=seqs)
+        assert_attn_close(out.cpu().numpy()[seqs], ref[seqs], name)
+        assert_lse_close(lse.cpu().numpy()[seqs], rlse[seqs])
+        assert c.stats[oda.ODA_STAT_ROWS].item() == 8 * sum(len(pos(b, n - 1))
+                                                             for b, n in enumerate(lens))
+    with pytest.raises(oda.OdaError):          # one more sequence is refused on the host
+        big = oda.make_kv(c.kc, c.vc, torch.cat([c.bt, c.bt[:1]]),
+                          torch.cat([c.seq_lens, c.seq_lens[:1]]))
+        oda.oda_decode_full(big, torch.cat([c.q, c.q[:1]]), SCALE,
+                            torch.zeros(1025, 16, 128, device="cuda"), c.ws)
+
+
 def test_local_equals_full_when_window_covers_history():
     """s + w = 260 covers t + 1 <= 260 tokens: the same visible set (bit-exact in the plan
     export), hence the same attention up to fp32 summation order (Local runs the cluster
