@@ -745,6 +745,16 @@ def run_oda(args, dist: Dist):
     # ---- phase breakdown: same graphs with event nodes at the phase boundaries ----
     result["phases"], step = phase_breakdown(s, w, theta, PH, step, stream)
     result["gate_cost"], step = gate_cost(s, w, theta, GC, step, stream)
+    # the two ends of the Full-call rate: every step Local only (rho = 0) and every step
+    # recomputed with Full (rho = 1), from the same interleaved timings
+    ctx = float(np.mean(s.lengths)) + step
+    T = result["gate_cost"]["ms_per_step"]
+    for name, key, rows in [("rho_0", "theta_plus_inf", min(ctx, w.sink + w.window)),
+                            ("rho_1", "theta_minus_inf", min(ctx, w.sink + w.window) + ctx)]:
+        kv = w.batch * w.layers * w.num_kv_heads * rows * ROW_BYTES
+        result[name] = {"tokens_per_s": w.batch / (T[key] / 1e3), "ms_per_step": T[key],
+                        "kv_gbs": kv / (T[key] / 1e3) / 1e9,
+                        "frac_of_peak": kv / (T[key] / 1e3) / 1e9 / peak}
     result["variants"], step = step_variants(s, w, theta, rho, VAR, step, stream)
 
     # ---- dominant kernel alone: Full decode at this context, CUDA events per launch ----

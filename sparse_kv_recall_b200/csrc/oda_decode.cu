@@ -598,6 +598,249 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Short-window kernel (Local at small batch). The split above ends a short launch with a
+// chain of global round trips: every CTA's partial to global memory, an acquire-release
+// ticket, the last CTA reading every partial back. Here one thread-block cluster of
+// kClusterCtas CTAs takes one (sequence, KV head); each of its kClusterCtas x kClusterWarps
+// warps attends at most one page, and the CTAs' partials are merged through distributed
+// shared memory by cluster rank 0 between two cluster barriers. The page step, the commit
+// of slot t and the in-CTA merge are those of decode_kernel.
+// ---------------------------------------------------------------------------------------
+constexpr int kClusterCtas = 8;
+constexpr int kClusterWarps = 17;
+constexpr int kClusterThreads = kClusterWarps * 32;
+constexpr int kClusterPages = kClusterCtas * kClusterWarps;  // pages per (b, g) at most
+
+template <int G>
+__global__ void __launch_bounds__(kClusterThreads, 1) cluster_decode_kernel(const DecodeParams p) {
+  constexpr int VPL = Vpl<G>::value;
+  constexpr int kPs = 18 * G;
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned char* stages = smem;  // [warp][kStageBytes]: one page per warp
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kClusterWarps * kStageBytes);
+  float* pscratch = reinterpret_cast<float*>(bars + kClusterWarps);  // [warp][kPs]
+  // rank 0's copy gathers every CTA's partial: [kClusterCtas][G * 128 outputs + G log-sums]
+  float* part = pscratch + kClusterWarps * kPs;
+  __shared__ unsigned long long s_rows, s_pages;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int half = lane >> 4, li = lane & 15;
+  const unsigned rank = cluster_ctarank();
+  const int bg = blockIdx.x / kClusterCtas;
+  const int b = bg / p.hkv, g = bg % p.hkv;
+  if (tid == 0) {
+    s_rows = 0;
+    s_pages = 0;
+  }
+  if (lane == 0) {
+    mbar_init(&bars[warp], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (p.wait_first) griddep_wait();
+
+  // Before the dependency wait: the plan and this warp's page copy (history pages only).
+  const SeqPlan sp = make_plan(p.plan, b);
+  if (rank == 0 && g == 0 && tid == 0 && sp.err != 0) report(p.status, sp.err);
+  const int j = (int)rank * kClusterWarps + warp;
+  const bool has = !sp.skip && j < sp.npages;
+  const size_t head_off = (size_t)g * (kPage * kHeadDim);
+  const size_t page_stride = (size_t)p.hkv * kPage * kHeadDim;
+  unsigned char* st = stages + warp * kStageBytes;
+  PageRef r;
+  r.err = 0;
+  r.lp = 0;
+  r.pb = 0;
+  if (has) {
+    r = page_ref(p.plan, sp, b, j);
+    if (lane == 0) {
+      if (r.err == 0) {
+        const uint64_t policy = l2_evict_first_policy();
+        const size_t src = (size_t)r.pb * page_stride + head_off;
+        mbar_arrive_expect_tx(&bars[warp], kStageBytes);
+        bulk_load(st, p.k_cache + src, kPageBytes, &bars[warp], policy);
+        bulk_load(st + kPageBytes, p.v_cache + src, kPageBytes, &bars[warp], policy);
+      } else {
+        report(p.status, r.err);
+      }
+    }
+  }
+  __syncwarp();
+  if (!p.wait_first) griddep_wait();
+  griddep_launch_dependents();
+
+  float m_run[VPL], l_run[VPL];
+  f2_t acc[G][4];
+#pragma unroll
+  for (int u = 0; u < VPL; ++u) {
+    m_run[u] = -INFINITY;
+    l_run[u] = 0.f;
+  }
+#pragma unroll
+  for (int gg = 0; gg < G; ++gg)
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) acc[gg][jj] = f2_pack(0.f, 0.f);
+  unsigned rows_vis = 0, pages_read = 0;
+  if (has && r.err == 0) {
+    f2_t q2[G][4];
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      const uint4 qv = *reinterpret_cast<const uint4*>(
+          p.q + ((size_t)b * p.hq + g * G + gg) * kHeadDim + 8 * li);
+      float qf[8];
+      unpack8(qv, qf);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        q2[gg][jj] = f2_pack(qf[2 * jj] * p.scale_log2, qf[2 * jj + 1] * p.scale_log2);
+    }
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[warp], 0u))) {
+      if (lane == 0) report(p.status, ODA_DEV_TIMEOUT);
+    } else {
+      if (p.k_new != nullptr && r.lp == sp.t / kPage) {
+        // Commit: the step's K/V take slot t, in the cache and in this page's copy.
+        const int row = sp.t % kPage;
+        const bool isk = lane < 16;
+        const uint4 v = *reinterpret_cast<const uint4*>(
+            (isk ? p.k_new : p.v_new) + ((size_t)b * p.hkv + g) * kHeadDim + 8 * li);
+        *reinterpret_cast<uint4*>(st + (isk ? 0 : kPageBytes) + row * kRowBytes + 16 * li) = v;
+        __nv_bfloat16* dst = (isk ? p.k_cache_w : p.v_cache_w) + (size_t)r.pb * page_stride +
+                             head_off + row * kHeadDim + 8 * li;
+        *reinterpret_cast<uint4*>(dst) = v;
+        __syncwarp();
+      }
+      page_step<G>(st, q2, m_run, l_run, acc, pscratch + warp * kPs, sp, r.lp, lane, rows_vis);
+      pages_read = 1;
+    }
+  }
+
+  // ---- merge the CTA's 2 x kClusterWarps half-warp states ----
+  float lsum[VPL];
+#pragma unroll
+  for (int u = 0; u < VPL; ++u) {
+    float v = l_run[u];
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    lsum[u] = v;
+  }
+  if (p.stats != nullptr && lane == 0 && pages_read) {
+    atomicAdd(&s_rows, (unsigned long long)rows_vis);
+    atomicAdd(&s_pages, (unsigned long long)pages_read);
+  }
+  __syncthreads();  // every warp is done with its page: stage memory becomes merge scratch
+  if (p.stats != nullptr && tid == 0) {
+    if (s_rows) atomicAdd(&p.stats[ODA_STAT_ROWS], s_rows);
+    if (s_pages) atomicAdd(&p.stats[ODA_STAT_PAGES], s_pages);
+  }
+  constexpr int kStates = 2 * kClusterWarps;
+  float* Mw = reinterpret_cast<float*>(stages);  // [kStates][G]
+  float* Lw = Mw + kStates * G;                  // [kStates][G]
+  float* Aw = Lw + kStates * G;                  // [kStates][G][128]
+  const int sidx = warp * 2 + half;
+  if (li < 2 && (G >= 2 || li == 0)) {
+#pragma unroll
+    for (int u = 0; u < VPL; ++u) {
+      const int gh = (G >= 2) ? ((li & 1) * (G / 2) + u) : 0;
+      Mw[sidx * G + gh] = m_run[u];
+      Lw[sidx * G + gh] = lsum[u];
+    }
+  }
+#pragma unroll
+  for (int gg = 0; gg < G; ++gg) {
+    float a[8];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) f2_unpack(acc[gg][jj], a[2 * jj], a[2 * jj + 1]);
+    float4* dst = reinterpret_cast<float4*>(Aw + (sidx * G + gg) * kHeadDim + 8 * li);
+    dst[0] = make_float4(a[0], a[1], a[2], a[3]);
+    dst[1] = make_float4(a[4], a[5], a[6], a[7]);
+  }
+  __syncthreads();
+  // The CTA partial, with every thread: warp gg finds head gg's maximum and each state's
+  // weight, then thread groups sum interleaved states for one (head, dim) each, and the
+  // groups' sums are added in fixed order.
+  constexpr int kOut = G * kHeadDim;
+  constexpr int kGroups = kClusterThreads / kOut;  // 4, 2 or 1 for G = 1, 2, 4
+  float* Wt = Aw + kStates * G * kHeadDim;         // [kStates][G] weights
+  float* ML = Wt + kStates * G;                    // [G] max, [G] weight-sum
+  float* red = ML + 2 * G;                         // [kGroups][kOut]
+  if (warp < G) {
+    const int gg = warp;
+    float M = -INFINITY;
+    for (int s2 = lane; s2 < kStates; s2 += 32) M = fmaxf(M, Mw[s2 * G + gg]);
+#pragma unroll
+    for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+    float L = 0.f;
+    for (int s2 = lane; s2 < kStates; s2 += 32) {
+      const float ms = Mw[s2 * G + gg];
+      const float wt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+      Wt[s2 * G + gg] = wt;
+      L = fmaf(wt, Lw[s2 * G + gg], L);
+    }
+#pragma unroll
+    for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o2);
+    if (lane == 0) {
+      ML[gg] = M;
+      ML[G + gg] = L;
+    }
+  }
+  __syncthreads();
+  if (tid < kGroups * kOut) {
+    const int o = tid % kOut, sg = tid / kOut;
+    const int gg = o / kHeadDim, d = o % kHeadDim;
+    float a = 0.f;
+    for (int s2 = sg; s2 < kStates; s2 += kGroups)
+      a = fmaf(Wt[s2 * G + gg], Aw[(s2 * G + gg) * kHeadDim + d], a);
+    red[sg * kOut + o] = a;
+  }
+  __syncthreads();
+  constexpr int kPart = kOut + G;
+  if (tid < kOut) {  // pushed straight into rank 0's shared memory
+    const int gg = tid / kHeadDim;
+    const float M = ML[gg], L = ML[G + gg];
+    float a = 0.f;
+#pragma unroll
+    for (int sg = 0; sg < kGroups; ++sg) a += red[sg * kOut + tid];
+    float* slot = part + rank * kPart;
+    dsmem_st(slot + tid, 0, (M == -INFINITY) ? 0.f : a / L);
+    if (tid % kHeadDim == 0)
+      dsmem_st(slot + kOut + gg, 0, (M == -INFINITY) ? -INFINITY : M + log2f(L));
+  }
+  cluster_sync();  // every CTA's partial has landed in rank 0's shared memory
+  if (rank == 0 && !sp.skip && tid < kHeadDim) {
+    float ls[G][kClusterCtas], os[G][kClusterCtas];
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg)
+#pragma unroll
+      for (int c = 0; c < kClusterCtas; ++c) {
+        ls[gg][c] = part[c * kPart + kOut + gg];
+        os[gg][c] = part[c * kPart + gg * kHeadDim + tid];
+      }
+    float o[G], l2[G];
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kClusterCtas; ++c) M = fmaxf(M, ls[gg][c]);
+      if (M == -INFINITY) {
+        o[gg] = 0.f;
+        l2[gg] = -INFINITY;
+      } else {
+        float L = 0.f, a = 0.f;
+#pragma unroll
+        for (int c = 0; c < kClusterCtas; ++c) {
+          const float w = (ls[gg][c] == -INFINITY) ? 0.f : exp2f(ls[gg][c] - M);
+          L += w;
+          a = fmaf(w, os[gg][c], a);
+        }
+        o[gg] = a / L;
+        l2[gg] = M + log2f(L);
+      }
+    }
+    write_final<G>(p, b, g, o, l2);
+  }
+}
+
 // Debug export of the same plan: mask[b][p] = 1 for every visible position p < max_tokens.
 __global__ void visible_mask_kernel(PlanArgs a, uint8_t* mask, int max_tokens, int* status) {
   const int b = blockIdx.x;
@@ -643,13 +886,21 @@ static WsLayout ws_layout(int batch, int hkv, int G, int grid) {
   return w;
 }
 
+static size_t cluster_smem_bytes(int G) {
+  return (size_t)kClusterWarps * kStageBytes + (size_t)kClusterWarps * sizeof(uint64_t) +
+         (size_t)kClusterWarps * 18 * G * sizeof(float) +
+         (size_t)kClusterCtas * (G * kHeadDim + G) * sizeof(float);
+}
+
 template <int G>
 static int prepare_decode_kernel(int device) {
   static bool done[64] = {false};
   if (device < 0 || device >= 64) return ODA_ERR_CUDA;
   if (done[device]) return ODA_OK;
   if (cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)decode_smem_bytes(G)) != cudaSuccess)
+                           (int)decode_smem_bytes(G)) != cudaSuccess ||
+      cudaFuncSetAttribute(cluster_decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)cluster_smem_bytes(G)) != cudaSuccess)
     return ODA_ERR_CUDA;
   done[device] = true;
   return ODA_OK;
@@ -721,6 +972,36 @@ static cudaError_t launch_decode_kernel(const DecodeParams& p, int grid, size_t 
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, decode_kernel<G>, p);
+}
+
+template <int G>
+static cudaError_t launch_cluster_kernel(const DecodeParams& p, int grid, cudaStream_t st,
+                                         bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kClusterThreads);
+  cfg.dynamicSmemBytes = cluster_smem_bytes(G);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kClusterCtas;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, cluster_decode_kernel<G>, p);
+}
+
+// The short-window kernel takes a launch when the rule bounds every sequence's page list by
+// one cluster's warps (Local: sink pages + window pages) and one cluster per (sequence, KV
+// head) fits the GPU in one wave at one CTA per SM.
+static bool use_cluster_kernel(const oda_kv* kv, const oda_visibility& vis, const DeviceInfo& di) {
+  if (vis.mode != ODA_MODE_LOCAL) return false;
+  const long long pages = (vis.sink + kPage - 1) / kPage + (long long)(vis.window - 1) / kPage + 2;
+  return pages <= kClusterPages &&
+         (long long)kv->batch * kv->num_kv_heads * kClusterCtas <= di.sms;
 }
 
 int check_visibility(const oda_kv* kv, const oda_visibility* v) {
@@ -829,19 +1110,24 @@ int launch_decode(const oda_kv* kv, const oda_visibility& vis, const void* q, in
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t smem = decode_smem_bytes(G);
+  const bool cluster = use_cluster_kernel(kv, vis, di);
+  const int cgrid = kv->batch * kv->num_kv_heads * kClusterCtas;
   cudaError_t e;
   switch (G) {
     case 1:
       if ((rc = prepare_decode_kernel<1>(di.device)) != ODA_OK) return rc;
-      e = launch_decode_kernel<1>(p, grid, smem, st, pdl != 0);
+      e = cluster ? launch_cluster_kernel<1>(p, cgrid, st, pdl != 0)
+                  : launch_decode_kernel<1>(p, grid, smem, st, pdl != 0);
       break;
     case 2:
       if ((rc = prepare_decode_kernel<2>(di.device)) != ODA_OK) return rc;
-      e = launch_decode_kernel<2>(p, grid, smem, st, pdl != 0);
+      e = cluster ? launch_cluster_kernel<2>(p, cgrid, st, pdl != 0)
+                  : launch_decode_kernel<2>(p, grid, smem, st, pdl != 0);
       break;
     default:
       if ((rc = prepare_decode_kernel<4>(di.device)) != ODA_OK) return rc;
-      e = launch_decode_kernel<4>(p, grid, smem, st, pdl != 0);
+      e = cluster ? launch_cluster_kernel<4>(p, cgrid, st, pdl != 0)
+                  : launch_decode_kernel<4>(p, grid, smem, st, pdl != 0);
       break;
   }
   return cuda_status(e);

@@ -80,6 +80,33 @@ def test_maximum_batch_local_and_full():
                             torch.zeros(1025, 16, 128, device="cuda"), c.ws)
 
 
+@pytest.mark.parametrize("G,lens,sink,window", [
+    (2, [1], 4, 2048), (2, [17], 4, 2048), (2, [2053], 4, 2048), (2, [40_000], 4, 2048),
+    (1, [5000, 33], 4, 2048), (4, [9001, 2052], 0, 2100), (2, [700, 6000], 20, 100),
+    (2, [3000], 7, 33)])
+def test_local_short_window_cluster_path(G, lens, sink, window):
+    """Small batches take the cluster kernel for Local (one cluster per (sequence, KV head),
+    one page per warp, partials merged in distributed shared memory): outputs, normalisers,
+    attended rows and the fused commit against the oracle."""
+    c = Case(lens, hq=8 * G, hkv=8, seed=90 + G + len(lens))
+    out, lse = c.out_buffers()
+    _run(c, lambda: oda.oda_decode_local(c.kv, c.q, sink, window, SCALE, out, c.ws,
+                                         k_new=c.k_new, v_new=c.v_new, lse=lse))
+    pos = lambda b, t: O.local_positions(t, sink, window)
+    ref, rlse = c.oracle(pos, commit=True)
+    assert_attn_close(out.cpu().numpy(), ref, "local cluster G=%d" % G)
+    assert_lse_close(lse.cpu().numpy(), rlse)
+    assert c.stats[oda.ODA_STAT_ROWS].item() == 8 * sum(len(pos(b, n - 1))
+                                                         for b, n in enumerate(lens))
+    old_k = c.kbits
+    c.snapshot()
+    for b, n in enumerate(lens):
+        assert np.array_equal(c.slot_bits(c.kbits, b, n - 1), c.knew_bits[b])
+    pages, _, rows, _ = np.nonzero(c.kbits != old_k)
+    slots = {(int(c.bt_h[b, (n - 1) // 16]), (n - 1) % 16) for b, n in enumerate(lens)}
+    assert set(zip(pages.tolist(), rows.tolist())) <= slots
+
+
 def test_local_equals_full_when_window_covers_history():
     """s + w = 260 covers t + 1 <= 260 tokens: the same visible set (bit-exact in the plan
     export), hence the same attention up to fp32 summation order (Local runs the cluster
