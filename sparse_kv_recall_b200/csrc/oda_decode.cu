@@ -607,13 +607,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
 // shared memory by cluster rank 0 between two cluster barriers. The page step, the commit
 // of slot t and the in-CTA merge are those of decode_kernel.
 // ---------------------------------------------------------------------------------------
-constexpr int kClusterCtas = 8;
-constexpr int kClusterWarps = 17;
+constexpr int kClusterCtas = 16;  // a non-portable cluster size (B200 supports 16)
+constexpr int kClusterWarps = 9;
 constexpr int kClusterThreads = kClusterWarps * 32;
 constexpr int kClusterPages = kClusterCtas * kClusterWarps;  // pages per (b, g) at most
 
 template <int G>
-__global__ void __launch_bounds__(kClusterThreads, 1) cluster_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kClusterThreads, 2) cluster_decode_kernel(const DecodeParams p) {
   constexpr int VPL = Vpl<G>::value;
   constexpr int kPs = 18 * G;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -760,7 +760,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) cluster_decode_kernel(cons
   // weight, then thread groups sum interleaved states for one (head, dim) each, and the
   // groups' sums are added in fixed order.
   constexpr int kOut = G * kHeadDim;
-  constexpr int kGroups = kClusterThreads / kOut;  // 4, 2 or 1 for G = 1, 2, 4
+  constexpr int kGroups = kClusterThreads / kOut > 0 ? kClusterThreads / kOut : 1;
   float* Wt = Aw + kStates * G * kHeadDim;         // [kStates][G] weights
   float* ML = Wt + kStates * G;                    // [G] max, [G] weight-sum
   float* red = ML + 2 * G;                         // [kGroups][kOut]
@@ -785,8 +785,8 @@ __global__ void __launch_bounds__(kClusterThreads, 1) cluster_decode_kernel(cons
     }
   }
   __syncthreads();
-  if (tid < kGroups * kOut) {
-    const int o = tid % kOut, sg = tid / kOut;
+  for (int i = tid; i < kGroups * kOut; i += kClusterThreads) {
+    const int o = i % kOut, sg = i / kOut;
     const int gg = o / kHeadDim, d = o % kHeadDim;
     float a = 0.f;
     for (int s2 = sg; s2 < kStates; s2 += kGroups)
@@ -795,15 +795,15 @@ __global__ void __launch_bounds__(kClusterThreads, 1) cluster_decode_kernel(cons
   }
   __syncthreads();
   constexpr int kPart = kOut + G;
-  if (tid < kOut) {  // pushed straight into rank 0's shared memory
-    const int gg = tid / kHeadDim;
+  for (int o = tid; o < kOut; o += kClusterThreads) {  // pushed into rank 0's shared memory
+    const int gg = o / kHeadDim;
     const float M = ML[gg], L = ML[G + gg];
     float a = 0.f;
 #pragma unroll
-    for (int sg = 0; sg < kGroups; ++sg) a += red[sg * kOut + tid];
+    for (int sg = 0; sg < kGroups; ++sg) a += red[sg * kOut + o];
     float* slot = part + rank * kPart;
-    dsmem_st(slot + tid, 0, (M == -INFINITY) ? 0.f : a / L);
-    if (tid % kHeadDim == 0)
+    dsmem_st(slot + o, 0, (M == -INFINITY) ? 0.f : a / L);
+    if (o % kHeadDim == 0)
       dsmem_st(slot + kOut + gg, 0, (M == -INFINITY) ? -INFINITY : M + log2f(L));
   }
   cluster_sync();  // every CTA's partial has landed in rank 0's shared memory
@@ -900,7 +900,9 @@ static int prepare_decode_kernel(int device) {
   if (cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)decode_smem_bytes(G)) != cudaSuccess ||
       cudaFuncSetAttribute(cluster_decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)cluster_smem_bytes(G)) != cudaSuccess)
+                           (int)cluster_smem_bytes(G)) != cudaSuccess ||
+      cudaFuncSetAttribute(cluster_decode_kernel<G>,
+                           cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
     return ODA_ERR_CUDA;
   done[device] = true;
   return ODA_OK;
@@ -996,12 +998,12 @@ static cudaError_t launch_cluster_kernel(const DecodeParams& p, int grid, cudaSt
 
 // The short-window kernel takes a launch when the rule bounds every sequence's page list by
 // one cluster's warps (Local: sink pages + window pages) and one cluster per (sequence, KV
-// head) fits the GPU in one wave at one CTA per SM.
+// head) fits the GPU in one wave at two CTAs per SM.
 static bool use_cluster_kernel(const oda_kv* kv, const oda_visibility& vis, const DeviceInfo& di) {
   if (vis.mode != ODA_MODE_LOCAL) return false;
   const long long pages = (vis.sink + kPage - 1) / kPage + (long long)(vis.window - 1) / kPage + 2;
   return pages <= kClusterPages &&
-         (long long)kv->batch * kv->num_kv_heads * kClusterCtas <= di.sms;
+         (long long)kv->batch * kv->num_kv_heads * kClusterCtas <= 2ll * di.sms;
 }
 
 int check_visibility(const oda_kv* kv, const oda_visibility* v) {
