@@ -756,55 +756,32 @@ __global__ void __launch_bounds__(kClusterThreads, 2) cluster_decode_kernel(cons
     dst[1] = make_float4(a[4], a[5], a[6], a[7]);
   }
   __syncthreads();
-  // The CTA partial, with every thread: warp gg finds head gg's maximum and each state's
-  // weight, then thread groups sum interleaved states for one (head, dim) each, and the
-  // groups' sums are added in fixed order.
+  // The CTA partial: one thread per (head, dim) output reads every state's max and sum
+  // (broadcast shared loads), weighs the states and pushes the normalised result and the
+  // log-sum straight into rank 0's shared memory.
   constexpr int kOut = G * kHeadDim;
-  constexpr int kGroups = kClusterThreads / kOut > 0 ? kClusterThreads / kOut : 1;
-  float* Wt = Aw + kStates * G * kHeadDim;         // [kStates][G] weights
-  float* ML = Wt + kStates * G;                    // [G] max, [G] weight-sum
-  float* red = ML + 2 * G;                         // [kGroups][kOut]
-  if (warp < G) {
-    const int gg = warp;
-    float M = -INFINITY;
-    for (int s2 = lane; s2 < kStates; s2 += 32) M = fmaxf(M, Mw[s2 * G + gg]);
-#pragma unroll
-    for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
-    float L = 0.f;
-    for (int s2 = lane; s2 < kStates; s2 += 32) {
-      const float ms = Mw[s2 * G + gg];
-      const float wt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-      Wt[s2 * G + gg] = wt;
-      L = fmaf(wt, Lw[s2 * G + gg], L);
-    }
-#pragma unroll
-    for (int o2 = 16; o2 >= 1; o2 >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o2);
-    if (lane == 0) {
-      ML[gg] = M;
-      ML[G + gg] = L;
-    }
-  }
-  __syncthreads();
-  for (int i = tid; i < kGroups * kOut; i += kClusterThreads) {
-    const int o = i % kOut, sg = i / kOut;
-    const int gg = o / kHeadDim, d = o % kHeadDim;
-    float a = 0.f;
-    for (int s2 = sg; s2 < kStates; s2 += kGroups)
-      a = fmaf(Wt[s2 * G + gg], Aw[(s2 * G + gg) * kHeadDim + d], a);
-    red[sg * kOut + o] = a;
-  }
-  __syncthreads();
   constexpr int kPart = kOut + G;
-  for (int o = tid; o < kOut; o += kClusterThreads) {  // pushed into rank 0's shared memory
-    const int gg = o / kHeadDim;
-    const float M = ML[gg], L = ML[G + gg];
-    float a = 0.f;
+  float* slot = part + rank * kPart;
+  for (int o = tid; o < kOut; o += kClusterThreads) {
+    const int gg = o / kHeadDim, d = o % kHeadDim;
+    float M = -INFINITY;
 #pragma unroll
-    for (int sg = 0; sg < kGroups; ++sg) a += red[sg * kOut + o];
-    float* slot = part + rank * kPart;
-    dsmem_st(slot + o, 0, (M == -INFINITY) ? 0.f : a / L);
-    if (o % kHeadDim == 0)
-      dsmem_st(slot + kOut + gg, 0, (M == -INFINITY) ? -INFINITY : M + log2f(L));
+    for (int s2 = 0; s2 < kStates; ++s2) M = fmaxf(M, Mw[s2 * G + gg]);
+    float oval = 0.f, l2 = -INFINITY;
+    if (M != -INFINITY) {
+      float L = 0.f, a = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < kStates; ++s2) {
+        const float ms = Mw[s2 * G + gg];
+        const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+        L = fmaf(w, Lw[s2 * G + gg], L);
+        a = fmaf(w, Aw[(s2 * G + gg) * kHeadDim + d], a);
+      }
+      oval = a / L;
+      l2 = M + log2f(L);
+    }
+    dsmem_st(slot + o, 0, oval);
+    if (d == 0) dsmem_st(slot + kOut + gg, 0, l2);
   }
   cluster_sync();  // every CTA's partial has landed in rank 0's shared memory
   if (rank == 0 && !sp.skip && tid < kHeadDim) {
