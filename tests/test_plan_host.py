@@ -16,11 +16,12 @@ ROOT = os.path.dirname(HERE)
 
 
 @pytest.fixture(scope="module")
-def probe(tmp_path_factory):
+def probe():
     nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
     if not os.path.exists(nvcc):
         pytest.skip("nvcc not available")
-    exe = str(tmp_path_factory.mktemp("plan") / "plan_probe")
+    os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+    exe = os.path.join(ROOT, "_build", "plan_probe")
     cmd = [nvcc, "-std=c++17", "-O1", "-I", os.path.join(ROOT, "include"), "-I",
            os.path.join(ROOT, "sparse_kv_recall_b200", "csrc"), os.path.join(HERE, "plan_probe.cu"),
            "-o", exe]
