@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -175,9 +176,15 @@ def measured_peak():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the decode kernel's sources with comments and blank lines removed, so that a
+    change of wording does not void the stored ncu counters but any code change does."""
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        h.update(open(os.path.join(ROOT, "sparse_kv_recall_b200", "csrc", name), "rb").read())
+        text = open(os.path.join(ROOT, "sparse_kv_recall_b200", "csrc", name)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
+        h.update("\n".join(lines).encode())
     return h.hexdigest()[:16]
 
 

@@ -117,7 +117,9 @@ int oda_kv_append(const oda_kv* kv, const void* k_new, const void* v_new,
 /* Local ([ODA] 접근 방법, decoding procedure; 주요 결과, last item): the first `sink`
  * positions plus the `window` most recent ones, the current position included, as a set
  * union. With non-null k_new / v_new (bf16 [batch][num_kv_heads][128]) the call also
- * commits them at slot t (as oda_kv_append would) and attends to them there. */
+ * commits them at slot t (as oda_kv_append would) and attends to them there. Small batches
+ * with short windows run on one thread-block cluster per (sequence, KV head); results agree
+ * with the split kernel to fp32 rounding (the summation order differs). */
 int oda_decode_local(const oda_kv* kv, const void* q, int32_t num_q_heads, int32_t sink,
                      int32_t window, float scale, const void* k_new, const void* v_new,
                      void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,

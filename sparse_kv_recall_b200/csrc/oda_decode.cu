@@ -12,6 +12,10 @@
 // memory; if the (b, g) spans several CTAs, each writes its normalised partial (O, log2-sum)
 // to the workspace and the last to arrive (atomic ticket) merges them in fixed order.
 //
+// Short windows at small batch (Local) take cluster_decode_kernel instead: one thread-block
+// cluster per (b, g), one page per warp, partials merged in distributed shared memory (see
+// that kernel). Both kernels share the plan, the page step and the commit of slot t.
+//
 // Lane layout for a 16 x 128 page: lane = 16 * half + li; lane li owns dims [8 li, 8 li + 8)
 // of rows 2k + half, k = 0..7. Dot products are reduced over the 16 lanes of a half by a
 // reduce-scatter butterfly, after which lane li holds row 2 (li / 2) + half for heads
