@@ -68,7 +68,7 @@ def parse_args():
                     help="Full kernels launch every step and skip ungated sequences on-device "
                          "instead of sitting behind a graph IF node (ncu can list kernel nodes "
                          "only of graphs without conditional nodes)")
-    ap.add_argument("--profile-kernel", choices=["full", "local", "recall"],
+    ap.add_argument("--profile-kernel", choices=["full", "local", "recall", "train"],
                     help="one layer of the workload, the named kernel launched --steps times "
                          "(a small case for ncu captures); prints nothing")
     return ap.parse_args()
@@ -970,14 +970,27 @@ def run_profile_case(args):
     qo = torch.empty(w.batch, dtype=torch.float32, device=dev)
     go = torch.empty(w.batch, dtype=torch.int32, device=dev)
     scale = 1.0 / math.sqrt(128)
+    if args.profile_kernel == "train":          # the recall head's loss and gradient, batch 8
+        wt = oda_synth.scaled(w, batch=8)
+        g = torch.Generator(device=dev).manual_seed(wt.seed)
+        x = [torch.randn(8, wt.hidden, generator=g, device=dev) for _ in range(3)]
+        gain = oda_synth.make_gains(wt, 0, device=dev)
+        tws = torch.zeros(oda.oda_recall_train_workspace_size(8, wt.hidden, wt.mlp),
+                          dtype=torch.uint8, device=dev)
+        loss, db2 = torch.empty(1, device=dev), torch.empty(1, device=dev)
+        dw1, db1, dw2 = torch.empty_like(rw.w1), torch.empty_like(rw.b1), torch.empty_like(rw.w2)
+        train = lambda: oda.oda_recall_loss_grad(*x, rw.w1, rw.b1, rw.w2, rw.b2, gain, 0.5, tws,
+                                                 loss, dw1, db1, dw2, db2)
     for _ in range(args.steps):
         if args.profile_kernel == "full":
             oda.oda_decode_full(kv, si.q_full[0], scale, out, ws)
         elif args.profile_kernel == "local":
             oda.oda_decode_local(kv, si.q_local[0], w.sink, w.window, scale, out, ws)
-        else:
+        elif args.profile_kernel == "recall":
             oda.oda_recall_score(h, si.emb, out.view(w.batch, -1), rw.w1, rw.b1, rw.w2, rw.b2,
                                  0.0, qo, go, rws)
+        else:
+            train()
     torch.cuda.synchronize()
 
 
