@@ -470,7 +470,7 @@ def cp_emulation(s, w, stream, reps: int = 10):
 
 
 def run_train_grad(w, dev, stream, batch: int = 8, reps: int = 50):
-    """Recall-head training objective: loss and gradient (oda_recall_loss_grad, three
+    """Recall-head training objective: loss and gradient (oda_recall_loss_grad, two
     launches) for a batch of `batch` rows at the workload's hidden size, timed over `reps`
     calls captured in one CUDA graph. Bytes: W1 read once, dW1 written once."""
     from sparse_kv_recall_b200 import oda
@@ -502,7 +502,7 @@ def run_train_grad(w, dev, stream, batch: int = 8, reps: int = 50):
     nbytes = 2 * rw.w1.numel() * 4
     del graph
     return {"batch": batch, "hidden": wl.hidden, "mlp": wl.mlp, "us_per_call": us,
-            "launches_per_call": 3, "w1_read_plus_dw1_write_bytes": nbytes,
+            "launches_per_call": 2, "w1_read_plus_dw1_write_bytes": nbytes,
             "gbs": nbytes / (us / 1e6) / 1e9, "loss": float(loss.item())}
 
 

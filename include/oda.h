@@ -263,8 +263,8 @@ int oda_recall_score(const float* h_prev, const float* emb, const void* h_local,
  * (fp32 scalar at loss_out) and its gradient with respect to the head's parameters:
  * dw1 fp32 [3 * hidden][mlp], db1 / dw2 fp32 [mlp], db2 fp32 [1]; all outputs are fully
  * overwritten. batch <= 1024; mlp a multiple of 64. ws: oda_recall_train_workspace_size()
- * bytes, zero-filled once before first use (its ticket is left zero, the rest is scratch).
- * Three kernel launches; deterministic. */
+ * bytes, zero-filled once before first use (its tickets are left zero, the rest is scratch).
+ * Two kernel launches; deterministic. */
 int oda_recall_train_workspace_size(int32_t batch, int32_t hidden, int32_t mlp, size_t* bytes);
 int oda_recall_loss_grad(const float* h_prev, const float* emb, const void* h_local,
                          int32_t h_local_dtype, int32_t batch, int32_t hidden, int32_t mlp,

@@ -4,11 +4,12 @@
 //   z = W1^T x + b1,  a = GELU(z),  q = w2 . a + b2,  r = q - y,  loss = mean_b Huber(r)
 //   dq_b = clip(r_b, -delta, delta) / B,  dw2 = sum_b dq_b a_b,  db2 = sum_b dq_b,
 //   dz_b = dq_b w2 * GELU'(z_b),  db1 = sum_b dz_b,  dW1 = sum_b x_b dz_b^T.
-// Three launches:
-//   1. train_z_kernel     (slab, column tile) CTAs stream W1 once: partial z per slab;
-//   2. train_head_kernel  one CTA per column tile: z, a, q partials; the last tile forms q,
+// Two launches:
+//   1. train_z_kernel     (slab, column tile) CTAs stream W1 once: partial z per slab; the
+//                         last slab CTA of each column tile (acquire-release ticket) forms
+//                         z, a and q partials for its columns; the last tile then forms q,
 //                         the targets, the loss, dq and db2;
-//   3. train_grad_kernel  one CTA per 32-row block of W1: dz for every column (recomputed
+//   2. train_grad_kernel  one CTA per 32-row block of W1: dz for every column (recomputed
 //                         from z and dq), then its rows of dW1 written once, coalesced; the
 //                         first CTA also writes db1 and dw2.
 // dW1 (3 hidden x mlp fp32) is written once and W1 read once: the pair bounds the time.
@@ -40,7 +41,7 @@ static TrainWs train_ws(int batch, int hidden, int mlp) {
   w.q_part_off = w.z_off + align_t((size_t)batch * mlp * sizeof(float));
   w.dq_off = w.q_part_off + align_t((size_t)w.tiles * batch * sizeof(float));
   w.ticket_off = w.dq_off + align_t((size_t)batch * sizeof(float));
-  w.total = w.ticket_off + align_t(sizeof(unsigned));
+  w.total = w.ticket_off + align_t((size_t)(w.tiles + 1) * sizeof(unsigned));
   return w;
 }
 
@@ -63,7 +64,7 @@ struct TrainParams {
   float* z;            // [batch][mlp], b1 included
   float* q_part;       // [tiles][batch]
   float* dq;           // [batch]
-  unsigned* ticket;
+  unsigned* tickets;   // [tiles + 1]
 };
 
 __device__ __forceinline__ float gelu_erf_grad(float z) {
@@ -74,23 +75,24 @@ __device__ __forceinline__ float gelu_erf_grad(float z) {
 __global__ void __launch_bounds__(kRThreads) train_z_kernel(const TrainParams p) {
   __shared__ float xs[kBTile][kRows];
   __shared__ float red[kRowGroups][kBTile][kColTile];
+  __shared__ float qs[kRowGroups][2];
+  __shared__ int s_last;
+  __shared__ float s_h[kMaxTrainBatch], s_dq[kMaxTrainBatch];
   const int tid = threadIdx.x;
   const int rg = tid / kColTile, col = tid % kColTile;
   const int slab = blockIdx.x, tile = blockIdx.y;
+  const int slabs = gridDim.x, tiles = gridDim.y;
   const int r0 = slab * kRows;
   const int nrows = min(kRows, 3 * p.hidden - r0);
   const int gcol = tile * kColTile + col;
   float wv[kRowsPerThread];
   load_w1_slab(p.w1, p.mlp, r0, nrows, gcol, rg, wv);
   slab_partial_z(p.in, wv, p.batch, p.mlp, slab, r0, nrows, gcol, xs, red, p.z_part);
-}
 
-__global__ void __launch_bounds__(kRThreads) train_head_kernel(const TrainParams p, int slabs) {
-  __shared__ float qs[kRowGroups][2];
-  __shared__ int s_last;
-  const int tid = threadIdx.x;
-  const int tile = blockIdx.x, tiles = gridDim.x;
-  const int gcol = tile * kColTile + tid % kColTile;
+  // ---- last slab of this column tile: z (stored for the gradient), GELU, w2 ----
+  if (tid == 0) s_last = ticket_arrive(&p.tickets[tile]) == (unsigned)(slabs - 1);
+  __syncthreads();
+  if (!s_last) return;
   const int bl = tid / kColTile;
   for (int b0 = 0; b0 < p.batch; b0 += kRowGroups) {
     const int b = b0 + bl;
@@ -108,12 +110,12 @@ __global__ void __launch_bounds__(kRThreads) train_head_kernel(const TrainParams
       p.q_part[(size_t)tile * p.batch + b0 + tid] = qs[tid][0] + qs[tid][1];
     __syncthreads();
   }
-  // the last column tile to finish forms q, the loss and dq
-  __syncthreads();
-  if (tid == 0) s_last = ticket_arrive(p.ticket) == (unsigned)(tiles - 1);
+  if (tid == 0) p.tickets[tile] = 0u;
+
+  // ---- last column tile: q, the loss and dq ----
+  if (tid == 0) s_last = ticket_arrive(&p.tickets[tiles]) == (unsigned)(tiles - 1);
   __syncthreads();
   if (!s_last) return;
-  __shared__ float s_h[kMaxTrainBatch], s_dq[kMaxTrainBatch];
   const float inv_b = 1.f / (float)p.batch;
   for (int b = tid; b < p.batch; b += kRThreads) {
     float q = 0.f;
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(kRThreads) train_head_kernel(const TrainParams
     }
     *p.loss_out = loss * inv_b;
     *p.db2 = db2;
-    *p.ticket = 0u;  // leave the workspace as found
+    p.tickets[tiles] = 0u;  // leave the workspace as found
   }
 }
 
@@ -247,10 +249,9 @@ extern "C" int oda_recall_loss_grad(const float* h_prev, const float* emb, const
   p.z = reinterpret_cast<float*>(w + wl.z_off);
   p.q_part = reinterpret_cast<float*>(w + wl.q_part_off);
   p.dq = reinterpret_cast<float*>(w + wl.dq_off);
-  p.ticket = reinterpret_cast<unsigned*>(w + wl.ticket_off);
+  p.tickets = reinterpret_cast<unsigned*>(w + wl.ticket_off);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   train_z_kernel<<<dim3(wl.slabs, wl.tiles), kRThreads, 0, st>>>(p);
-  train_head_kernel<<<wl.tiles, kRThreads, 0, st>>>(p, wl.slabs);
   train_grad_kernel<<<(3 * hidden + kGradRows - 1) / kGradRows, kRThreads, 0, st>>>(p);
   return cuda_status(cudaGetLastError());
 }
