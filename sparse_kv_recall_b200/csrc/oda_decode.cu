@@ -873,6 +873,10 @@ static size_t cluster_smem_bytes(int G) {
          (size_t)kClusterCtas * (G * kHeadDim + G) * sizeof(float);
 }
 
+// Clusters of the short-window kernel the device can hold at once, per device and group
+// size (0: the cluster shape cannot be scheduled here, e.g. under a partitioned GPU).
+static int g_max_clusters[64][kMaxGroup + 1];
+
 template <int G>
 static int prepare_decode_kernel(int device) {
   static bool done[64] = {false};
@@ -885,6 +889,23 @@ static int prepare_decode_kernel(int device) {
       cudaFuncSetAttribute(cluster_decode_kernel<G>,
                            cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
     return ODA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kClusterCtas);
+  cfg.blockDim = dim3(kClusterThreads);
+  cfg.dynamicSmemBytes = cluster_smem_bytes(G);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kClusterCtas;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, cluster_decode_kernel<G>, &cfg) != cudaSuccess) {
+    cudaGetLastError();  // not fatal: the split kernel serves every launch
+    n = 0;
+  }
+  g_max_clusters[device][G] = n;
   done[device] = true;
   return ODA_OK;
 }
@@ -980,11 +1001,13 @@ static cudaError_t launch_cluster_kernel(const DecodeParams& p, int grid, cudaSt
 // The short-window kernel takes a launch when the rule bounds every sequence's page list by
 // one cluster's warps (Local: sink pages + window pages) and one cluster per (sequence, KV
 // head) fits the GPU in one wave at two CTAs per SM.
-static bool use_cluster_kernel(const oda_kv* kv, const oda_visibility& vis, const DeviceInfo& di) {
+static bool use_cluster_kernel(const oda_kv* kv, const oda_visibility& vis, const DeviceInfo& di,
+                               int G) {
   if (vis.mode != ODA_MODE_LOCAL) return false;
   const long long pages = (vis.sink + kPage - 1) / kPage + (long long)(vis.window - 1) / kPage + 2;
-  return pages <= kClusterPages &&
-         (long long)kv->batch * kv->num_kv_heads * kClusterCtas <= 2ll * di.sms;
+  const long long clusters = (long long)kv->batch * kv->num_kv_heads;
+  return pages <= kClusterPages && clusters * kClusterCtas <= 2ll * di.sms &&
+         clusters <= g_max_clusters[di.device][G];
 }
 
 int check_visibility(const oda_kv* kv, const oda_visibility* v) {
@@ -1093,22 +1116,25 @@ int launch_decode(const oda_kv* kv, const oda_visibility& vis, const void* q, in
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t smem = decode_smem_bytes(G);
-  const bool cluster = use_cluster_kernel(kv, vis, di);
+  switch (G) {  // attributes and the cluster capacity first
+    case 1: rc = prepare_decode_kernel<1>(di.device); break;
+    case 2: rc = prepare_decode_kernel<2>(di.device); break;
+    default: rc = prepare_decode_kernel<4>(di.device); break;
+  }
+  if (rc != ODA_OK) return rc;
+  const bool cluster = use_cluster_kernel(kv, vis, di, G);
   const int cgrid = kv->batch * kv->num_kv_heads * kClusterCtas;
   cudaError_t e;
   switch (G) {
     case 1:
-      if ((rc = prepare_decode_kernel<1>(di.device)) != ODA_OK) return rc;
       e = cluster ? launch_cluster_kernel<1>(p, cgrid, st, pdl != 0)
                   : launch_decode_kernel<1>(p, grid, smem, st, pdl != 0);
       break;
     case 2:
-      if ((rc = prepare_decode_kernel<2>(di.device)) != ODA_OK) return rc;
       e = cluster ? launch_cluster_kernel<2>(p, cgrid, st, pdl != 0)
                   : launch_decode_kernel<2>(p, grid, smem, st, pdl != 0);
       break;
     default:
-      if ((rc = prepare_decode_kernel<4>(di.device)) != ODA_OK) return rc;
       e = cluster ? launch_cluster_kernel<4>(p, cgrid, st, pdl != 0)
                   : launch_decode_kernel<4>(p, grid, smem, st, pdl != 0);
       break;
