@@ -98,12 +98,14 @@ __device__ __forceinline__ float sum_slabs(const float* z_part, int b, int gcol,
   const size_t sstride = (size_t)batch * mlp;
   float z = 0.f;
   for (int s0 = 0; s0 < slabs; s0 += kSlabChunk) {
+    // every load unconditional (a clamped slab index past the end), so all of them issue
+    // back to back; the out-of-range ones are dropped from the sum
     float part[kSlabChunk];
 #pragma unroll
     for (int u = 0; u < kSlabChunk; ++u)
-      part[u] = (s0 + u < slabs) ? __ldcg(zp + (size_t)(s0 + u) * sstride) : 0.f;
+      part[u] = __ldcg(zp + (size_t)min(s0 + u, slabs - 1) * sstride);
 #pragma unroll
-    for (int u = 0; u < kSlabChunk; ++u) z += part[u];
+    for (int u = 0; u < kSlabChunk; ++u) z += (s0 + u < slabs) ? part[u] : 0.f;
   }
   return z;
 }
