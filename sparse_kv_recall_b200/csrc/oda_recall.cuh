@@ -61,12 +61,16 @@ __device__ __forceinline__ void slab_partial_z(const RecallInputs& in,
                                                float* z_part) {
   const int tid = threadIdx.x;
   const int rg = tid / kColTile, col = tid % kColTile;
+  static_assert(kRows == kRThreads, "each thread stages one row of the slab");
   for (int b0 = 0; b0 < batch; b0 += kBTile) {
     const int nb = min(kBTile, batch - b0);
-    for (int i = tid; i < nb * kRows; i += kRThreads) {
-      const int bb = i / kRows, r = i % kRows;
-      xs[bb][r] = r < nrows ? x_at(in, b0 + bb, r0 + r) : 0.f;
-    }
+    // thread tid stages row tid of every sequence of the tile, all loads in flight together
+    float xv[kBTile];
+#pragma unroll
+    for (int bb = 0; bb < kBTile; ++bb)
+      xv[bb] = (bb < nb && tid < nrows) ? x_at(in, b0 + bb, r0 + tid) : 0.f;
+#pragma unroll
+    for (int bb = 0; bb < kBTile; ++bb) xs[bb][tid] = xv[bb];
     __syncthreads();
     // only the nb sequences present (a batch of one does 1/8 of the FMAs of a full tile)
 #pragma unroll

@@ -159,6 +159,15 @@ __global__ void __launch_bounds__(kRThreads) train_grad_kernel(const TrainParams
     float db1 = 0.f, dw2 = 0.f;
     for (int b0 = 0; b0 < p.batch; b0 += kBTile) {
       const int nb = min(kBTile, p.batch - b0);
+      // this column's z and every dq of the tile, all loads issued together (clamped
+      // indices; rows past the batch are never used)
+      float zv[kBTile], dqv[kBTile];
+#pragma unroll
+      for (int bb = 0; bb < kBTile; ++bb) {
+        const int b = b0 + min(bb, nb - 1);
+        zv[bb] = has_c ? __ldcg(&p.z[(size_t)b * p.mlp + c]) : 0.f;
+        dqv[bb] = __ldcg(&p.dq[b]);
+      }
       __syncthreads();
       {  // one x value per thread: kBTile x kGradRows = 256
         const int bb = tid / kGradRows, i = tid % kGradRows;
@@ -168,9 +177,8 @@ __global__ void __launch_bounds__(kRThreads) train_grad_kernel(const TrainParams
 #pragma unroll
       for (int bb = 0; bb < kBTile; ++bb) {
         if (bb < nb && has_c) {
-          const int b = b0 + bb;
-          const float z = p.z[(size_t)b * p.mlp + c];
-          const float dq = p.dq[b];
+          const float z = zv[bb];
+          const float dq = dqv[bb];
           const float dz = dq * w2c * gelu_erf_grad(z);
           db1 += dz;
           dw2 = fmaf(dq, gelu_erf(z), dw2);
