@@ -180,3 +180,36 @@ def test_recall_training_argument_checks(lib):
     assert call(batch=2000) == I
     assert call(ws_bytes=16) == oda.ODA_ERR_WORKSPACE_TOO_SMALL
     assert call(batch=0) == oda.ODA_OK
+
+
+def test_step_desc_checks_before_any_cuda_call(lib):
+    """Per-layer access range, gate source and rho are validated on the host."""
+    I = oda.ODA_ERR_INVALID_ARG
+    L = 2
+    kvs = (oda.oda_kv * L)(_kv(), _kv())
+    P = ctypes.c_void_p
+    arr = lambda: (P * L)(0x1000, 0x2000)
+    keep = []
+
+    def desc(**kw):
+        a = [arr() for _ in range(7)]
+        keep.extend(a)
+        base = dict(num_layers=L, layers=ctypes.cast(kvs, ctypes.POINTER(oda.oda_kv)),
+                    num_q_heads=16, sink=4, window=256, scale=0.088,
+                    q_local=ctypes.cast(a[0], ctypes.POINTER(P)),
+                    k_local=ctypes.cast(a[1], ctypes.POINTER(P)),
+                    v_local=ctypes.cast(a[2], ctypes.POINTER(P)),
+                    q_full=ctypes.cast(a[3], ctypes.POINTER(P)),
+                    k_full=ctypes.cast(a[4], ctypes.POINTER(P)),
+                    v_full=ctypes.cast(a[5], ctypes.POINTER(P)),
+                    out=ctypes.cast(a[6], ctypes.POINTER(P)), mlp=256)
+        base.update(kw)
+        return oda.oda_step_desc(**base)
+
+    h = ctypes.c_void_p(0)
+    ints = lambda *v: ctypes.cast((ctypes.c_int32 * L)(*v), ctypes.POINTER(ctypes.c_int32))
+    for d in [desc(sinks=ints(4, -1)), desc(windows=ints(0, 256)), desc(window=0),
+              desc(gate_source=7), desc(gate_source=oda.ODA_GATE_RANDOM, gate_u=None, rho=0.5),
+              desc(gate_source=oda.ODA_GATE_RANDOM, gate_u=0x3000, rho=1.5)]:
+        assert lib.oda_step_graph_create(ctypes.byref(d), None, ctypes.byref(h)) == I
+        assert not h.value
