@@ -42,7 +42,7 @@ def _check(c, run, positions_of, seqs, commit=False):
     return out
 
 
-@pytest.mark.parametrize("seed", range(24))
+@pytest.mark.parametrize("seed", range(60))
 def test_random_rules_match_oracle(seed):
     r = np.random.default_rng(1000 + seed)
     c = _case(r, 500 + seed)
