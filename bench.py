@@ -42,6 +42,7 @@ DEFAULT_WORKLOAD = "qwen3-1.7b-128k-b1"
 ROW_BYTES = 2 * 128 * 2          # K row + V row of one (position, KV head): 512 B
 PAGE_BYTES = 2 * 16 * 128 * 2    # K page + V page of one (page, KV head): 8 KB
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0         # B200 HBM3e nominal (~8 TB/s), reported beside the measured peak
 PROFILE = os.path.join(ROOT, "profiles", "decode_full_128k.md")
 KERNEL_SOURCES = ["oda_decode.cu", "oda_plan.cuh", "oda_common.cuh"]
 
@@ -653,7 +654,9 @@ def run_da_main(args, dist: Dist, w, dev: str):
                       "modes": "global/focus/local p=%s" % (w.da_probs,), "kv_dtype": "bf16",
                       "l2": "no flush: ~1.9 GB of kept pages per step >> L2"},
            "kv_stream": {"gbs": r["kv_gbs"], "frac_of_peak": r["kv_gbs"] / peak, "peak_gbs": peak,
-                         "peak_kind": peak_kind, "attended_rows_per_step": r["attended_rows_per_step"]},
+                         "peak_kind": peak_kind, "frac_of_nominal": r["kv_gbs"] / NOMINAL_HBM_GBS,
+                         "nominal_gbs": NOMINAL_HBM_GBS,
+                         "attended_rows_per_step": r["attended_rows_per_step"]},
            "gpu_launches": r["gpu_launches"], "clocks": clocks.stop()}
     if "e2e" in r:
         res["e2e"] = {"value": r["e2e"]["tokens_per_s"], "unit": UNIT,
@@ -742,7 +745,9 @@ def run_oda(args, dist: Dist):
                    "parallelism": "replicas (dp%d, no collective)" % dist.world},
         "kv_stream": {"attended_bytes": kv_bytes, "gbs": kv_bytes / (ms_local / 1e3) / 1e9,
                       "frac_of_peak": kv_bytes / (ms_local / 1e3) / 1e9 / peak,
-                      "page_bytes": page_bytes, "peak_gbs": peak, "peak_kind": peak_kind},
+                      "page_bytes": page_bytes, "peak_gbs": peak, "peak_kind": peak_kind,
+                      "frac_of_nominal": kv_bytes / (ms_local / 1e3) / 1e9 / NOMINAL_HBM_GBS,
+                      "nominal_gbs": NOMINAL_HBM_GBS},
         "gpu_launches": launches,
         "clocks": clk,
     }
@@ -799,7 +804,8 @@ def run_oda(args, dist: Dist):
                           "frac": achieved / peak, "traffic": traffic,
                           "algorithmic_bytes": alg, "ms_per_launch": ms_launch, "timed": how,
                           "achieved_alone": achieved_alone, "frac_alone": achieved_alone / peak,
-                          "ms_per_launch_alone": dur, "peak_kind": peak_kind + " (copy)"}
+                          "ms_per_launch_alone": dur, "peak_kind": peak_kind + " (copy)",
+                          "frac_of_nominal": achieved / NOMINAL_HBM_GBS}
 
     if w.name == DEFAULT_WORKLOAD:
         result["context_parallel_1gpu"] = cp_emulation(s, w, stream)
