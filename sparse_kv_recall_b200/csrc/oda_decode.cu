@@ -194,6 +194,140 @@ __device__ __forceinline__ void page_step(const unsigned char* stage, const f2_t
   __syncwarp();
 }
 
+// ---- G = 4: page scores on the tensor cores ------------------------------------------
+// With four query heads per KV head the CUDA-core page step above is bound by instruction
+// issue (about twice the FMAs of G = 2 and a 32-value reduce-scatter), so decode_kernel<4>
+// forms the scores with mma.sync m16n8k16 (bf16 operands, fp32 accumulation; the products of
+// two bf16 values are exact in fp32): A = the page's 16 K rows, B = the group's query heads
+// as 8 columns (columns 4..7 zero), C = 16 tokens x 8 heads, eight k-steps of 16 dims.
+// Lane (gid = lane / 4, tig = lane % 4) supplies tokens gid and gid + 8 and the 16-byte dim
+// chunks tig + 4 j (j < 4) of them. Inside a chunk the k order is chosen so that each A and B
+// register is one 32-bit word of those chunks: k-step 2 j + h takes words 2 h and 2 h + 1 of
+// chunk tig + 4 j (rows gid and gid + 8 for A, head gid for B). No shuffles or transposes;
+// the 16-byte shared loads of a quarter-warp hit at most two lanes per bank group. The lane
+// then holds the scores of tokens gid and gid + 8 for heads 2 tig and 2 tig + 1; softmax
+// weights go to the same shared exchange as above and P.V stays on the CUDA cores.
+template <int G>
+struct MmaScores {
+  static constexpr bool value = G == 4;
+};
+
+__device__ __forceinline__ void mma_16816_bf16(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The query of head gid of group (b, g) as B fragments: chunks tig + 4 j, zero for gid >= G.
+template <int G>
+__device__ __forceinline__ void load_q_mma(const __nv_bfloat16* q, int lane, uint4 (&qv)[4]) {
+  const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    qv[j] = gid < G ? *reinterpret_cast<const uint4*>(q + gid * kHeadDim + 8 * (tig + 4 * j))
+                    : make_uint4(0u, 0u, 0u, 0u);
+}
+
+// A group's running maximum is raised only when a score exceeds it by more than this many
+// base-2 units, so the rescale of the accumulators is rare; unnormalised weights stay below
+// 2^kLazyMax, far inside fp32 range. (m, l, acc) keep their meaning: acc and l are sums of
+// 2^(s - m) with m the same for every lane that holds a head.
+constexpr float kLazyMax = 8.f;
+
+// One page for G = 4. m_run[u], l_run[u] belong to head 2 tig + u (l_run: this lane's tokens
+// only); acc is the half-warp P.V layout of page_step.
+template <int G>
+__device__ __forceinline__ void page_step_mma(const unsigned char* stage, const uint4 (&qv)[4],
+                                              float scale_log2, float (&m_run)[2],
+                                              float (&l_run)[2], f2_t (&acc)[G][4], float* ps,
+                                              const SeqPlan& sp, int lp, int lane,
+                                              unsigned& rows_vis) {
+  static_assert(G == 4, "tensor-core scores serve four heads per KV head");
+  const int gid = lane >> 2, tig = lane & 3;
+  const unsigned char* k0 = stage + gid * kRowBytes + 16 * tig;
+  const unsigned char* k1 = k0 + 8 * kRowBytes;
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 ka = *reinterpret_cast<const uint4*>(k0 + 64 * j);
+    const uint4 kb = *reinterpret_cast<const uint4*>(k1 + 64 * j);
+    mma_16816_bf16(c, ka.x, kb.x, ka.y, kb.y, qv[j].x, qv[j].y);
+    mma_16816_bf16(c, ka.z, kb.z, ka.w, kb.w, qv[j].z, qv[j].w);
+  }
+  const bool v0 = row_visible(sp, lp * kPage + gid);
+  const bool v1 = row_visible(sp, lp * kPage + gid + 8);
+  rows_vis += __popc(__ballot_sync(0xffffffffu, v0) & 0x11111111u) +
+              __popc(__ballot_sync(0xffffffffu, v1) & 0x11111111u);
+  const bool head_ok = 2 * tig < G;  // columns 2 tig, 2 tig + 1 are real heads
+  float s[2][2];                     // [token gid, gid + 8][head 2 tig + u]
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    s[0][u] = v0 ? c[u] * scale_log2 : -INFINITY;
+    s[1][u] = v1 ? c[2 + u] * scale_log2 : -INFINITY;
+  }
+  float* pshare = ps;           // [2 halves][8 rows][G], as page_step
+  float* ashare = ps + 16 * G;  // [G] rescale factors (written when a maximum is raised)
+  bool raise = false;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) raise |= head_ok && fmaxf(s[0][u], s[1][u]) > m_run[u] + kLazyMax;
+  const bool raised = __any_sync(0xffffffffu, raise);
+  if (raised) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float mx = fmaxf(s[0][u], s[1][u]);  // page maximum of the head over the 8 gid lanes
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const bool up = mx > m_run[u] + kLazyMax;
+      const float al = !up ? 1.f : (m_run[u] == -INFINITY ? 0.f : exp2f(m_run[u] - mx));
+      if (up) m_run[u] = mx;
+      l_run[u] *= al;
+      if (head_ok && gid == 0) ashare[2 * tig + u] = al;
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int r = gid + 8 * t;
+    const int slot = (r & 1) * 8 + (r >> 1);  // page_step's [half][k] order of row r
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float pr = (s[t][u] == -INFINITY) ? 0.f : exp2f(s[t][u] - m_run[u]);
+      l_run[u] += pr;
+      if (head_ok) pshare[slot * G + 2 * tig + u] = pr;
+    }
+  }
+  __syncwarp();
+
+  const int half = lane >> 4, li = lane & 15;
+  if (raised) {
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      const float al = ashare[gg];
+      const f2_t al2 = f2_pack(al, al);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[gg][j] = f2_mul(acc[gg][j], al2);
+    }
+  }
+  const uint4* V = reinterpret_cast<const uint4*>(stage + kPageBytes);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint4 vw = V[(2 * k + half) * 16 + li];
+    const f2_t vp[4] = {bf16x2_widen(vw.x), bf16x2_widen(vw.y), bf16x2_widen(vw.z),
+                        bf16x2_widen(vw.w)};
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      const float pk = pshare[(half * 8 + k) * G + gg];
+      const f2_t pp = f2_pack(pk, pk);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[gg][j] = f2_fma(pp, vp[j], acc[gg][j]);
+    }
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ void store_out(const DecodeParams& p, size_t idx, float v) {
   if (p.out_bf16)
     reinterpret_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
@@ -372,16 +506,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     __syncwarp();
     dep_wait();
 
-    f2_t q2[G][4];
+    f2_t q2[G][4];  // CUDA-core scores: scaled query dims 8 li .. 8 li + 7 of every head
+    uint4 qv[4];    // tensor-core scores: B fragments
+    if constexpr (MmaScores<G>::value) {
+      load_q_mma<G>(p.q + ((size_t)b * p.hq + g * G) * kHeadDim, lane, qv);
+    } else {
 #pragma unroll
-    for (int gg = 0; gg < G; ++gg) {
-      const uint4 qv = *reinterpret_cast<const uint4*>(
-          p.q + ((size_t)b * p.hq + g * G + gg) * kHeadDim + 8 * li);
-      float qf[8];
-      unpack8(qv, qf);
+      for (int gg = 0; gg < G; ++gg) {
+        const uint4 qw = *reinterpret_cast<const uint4*>(
+            p.q + ((size_t)b * p.hq + g * G + gg) * kHeadDim + 8 * li);
+        float qf[8];
+        unpack8(qw, qf);
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        q2[gg][j] = f2_pack(qf[2 * j] * p.scale_log2, qf[2 * j + 1] * p.scale_log2);
+        for (int j = 0; j < 4; ++j)
+          q2[gg][j] = f2_pack(qf[2 * j] * p.scale_log2, qf[2 * j + 1] * p.scale_log2);
+      }
     }
 
     for (int n = 0; n < cnt && !dead; ++n) {
@@ -413,7 +552,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
           fence_proxy_async_smem();  // this stage is refilled by a bulk copy later
           __syncwarp();
         }
-        page_step<G>(st, q2, m_run, l_run, acc, ps, sp, r.lp, lane, rows_vis);
+        if constexpr (MmaScores<G>::value)
+          page_step_mma<G>(st, qv, p.scale_log2, m_run, l_run, acc, ps, sp, r.lp, lane, rows_vis);
+        else
+          page_step<G>(st, q2, m_run, l_run, acc, ps, sp, r.lp, lane, rows_vis);
         ++pages_read;
       }
       __syncwarp();
@@ -423,13 +565,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     wcount += cnt;
 
     // ---- merge the 8 half-warp states of this piece ----
+    // State (warp, half) covers the page rows of parity `half`. Its softmax sum is spread over
+    // the lanes that scored those rows: li bits 1..3 of a half (CUDA-core scores), or gid bits
+    // 1..2 at a fixed gid parity and tig (tensor-core scores).
     float lsum[VPL];
 #pragma unroll
     for (int u = 0; u < VPL; ++u) {
       float v = l_run[u];
-      v += __shfl_xor_sync(0xffffffffu, v, 8);
-      v += __shfl_xor_sync(0xffffffffu, v, 4);
-      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      if constexpr (MmaScores<G>::value) {
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+      } else {
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+      }
       lsum[u] = v;
     }
     if (p.stats != nullptr && lane == 0 && (rows_vis | pages_read)) {
@@ -450,7 +600,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     float* Lw = Mw + 2 * kWarps * G;               // [2 * kWarps][G]
     float* Aw = Lw + 2 * kWarps * G;               // [2 * kWarps][G][128]
     const int sidx = warp * 2 + half;
-    if (li < 2 && (G >= 2 || li == 0)) {
+    if constexpr (MmaScores<G>::value) {
+      const int gid = lane >> 2, tig = lane & 3;  // lane gid < 2 holds rows of parity gid
+      if (gid < 2 && 2 * tig < G) {
+#pragma unroll
+        for (int u = 0; u < VPL; ++u) {
+          Mw[(warp * 2 + gid) * G + 2 * tig + u] = m_run[u];
+          Lw[(warp * 2 + gid) * G + 2 * tig + u] = lsum[u];
+        }
+      }
+    } else if (li < 2 && (G >= 2 || li == 0)) {
 #pragma unroll
       for (int u = 0; u < VPL; ++u) {
         const int gh = (G >= 2) ? ((li & 1) * (G / 2) + u) : 0;
