@@ -14,12 +14,13 @@
 //
 // Short windows at small batch (Local) take cluster_decode_kernel instead: one thread-block
 // cluster per (b, g), one page per warp, partials merged in distributed shared memory (see
-// that kernel). Both kernels share the plan, the page step and the commit of slot t.
+// that kernel). Both kernels share the plan, the P.V step and the commit of slot t.
 //
 // Lane layout for a 16 x 128 page: lane = 16 * half + li; lane li owns dims [8 li, 8 li + 8)
-// of rows 2k + half, k = 0..7. Dot products are reduced over the 16 lanes of a half by a
-// reduce-scatter butterfly, after which lane li holds row 2 (li / 2) + half for heads
-// (li % 2) * G / 2 + u.
+// of rows 2k + half, k = 0..7, for P.V. The CUDA-core scores (cluster_decode_kernel, and
+// decode_kernel<1>) are reduced over the 16 lanes of a half by a reduce-scatter butterfly,
+// after which lane li holds row 2 (li / 2) + half for heads (li % 2) * G / 2 + u;
+// decode_kernel<2> and <4> form the scores on the tensor cores (page_step_mma).
 #include <math.h>
 
 #include "oda_internal.h"
@@ -194,12 +195,13 @@ __device__ __forceinline__ void page_step(const unsigned char* stage, const f2_t
   __syncwarp();
 }
 
-// ---- G = 4: page scores on the tensor cores ------------------------------------------
+// ---- G = 2, 4: page scores on the tensor cores -----------------------------------------
 // With four query heads per KV head the CUDA-core page step above is bound by instruction
 // issue (about twice the FMAs of G = 2 and a 32-value reduce-scatter), so decode_kernel<4>
-// forms the scores with mma.sync m16n8k16 (bf16 operands, fp32 accumulation; the products of
-// two bf16 values are exact in fp32): A = the page's 16 K rows, B = the group's query heads
-// as 8 columns (columns 4..7 zero), C = 16 tokens x 8 heads, eight k-steps of 16 dims.
+// and decode_kernel<2> form the scores with mma.sync m16n8k16 (bf16 operands, fp32
+// accumulation; the products of two bf16 values are exact in fp32): A = the page's 16 K rows,
+// B = the group's query heads as 8 columns (columns G..7 zero), C = 16 tokens x 8 heads,
+// eight k-steps of 16 dims.
 // Lane (gid = lane / 4, tig = lane % 4) supplies tokens gid and gid + 8 and the 16-byte dim
 // chunks tig + 4 j (j < 4) of them. Inside a chunk the k order is chosen so that each A and B
 // register is one 32-bit word of those chunks: k-step 2 j + h takes words 2 h and 2 h + 1 of
@@ -209,7 +211,7 @@ __device__ __forceinline__ void page_step(const unsigned char* stage, const f2_t
 // weights go to the same shared exchange as above and P.V stays on the CUDA cores.
 template <int G>
 struct MmaScores {
-  static constexpr bool value = G == 4;
+  static constexpr bool value = G == 4 || G == 2;
 };
 
 __device__ __forceinline__ void mma_16816_bf16(float (&c)[4], uint32_t a0, uint32_t a1,
@@ -237,15 +239,16 @@ __device__ __forceinline__ void load_q_mma(const __nv_bfloat16* q, int lane, uin
 // 2^(s - m) with m the same for every lane that holds a head.
 constexpr float kLazyMax = 8.f;
 
-// One page for G = 4. m_run[u], l_run[u] belong to head 2 tig + u (l_run: this lane's tokens
-// only); acc is the half-warp P.V layout of page_step.
+// One page for G = 2 or 4. m_run[u], l_run[u] belong to head 2 tig + u (l_run: this lane's
+// tokens only; lanes with 2 tig >= G hold no head); acc is the half-warp P.V layout of
+// page_step.
 template <int G>
 __device__ __forceinline__ void page_step_mma(const unsigned char* stage, const uint4 (&qv)[4],
                                               float scale_log2, float (&m_run)[2],
                                               float (&l_run)[2], f2_t (&acc)[G][4], float* ps,
                                               const SeqPlan& sp, int lp, int lane,
                                               unsigned& rows_vis) {
-  static_assert(G == 4, "tensor-core scores serve four heads per KV head");
+  static_assert(G == 4 || G == 2, "tensor-core scores serve two or four heads per KV head");
   const int gid = lane >> 2, tig = lane & 3;
   const unsigned char* k0 = stage + gid * kRowBytes + 16 * tig;
   const unsigned char* k1 = k0 + 8 * kRowBytes;
@@ -356,7 +359,7 @@ __device__ __forceinline__ int cta_of(long long x, long long T, int P) {
 
 template <int G>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecodeParams p) {
-  constexpr int VPL = Vpl<G>::value;
+  constexpr int VPL = MmaScores<G>::value ? 2 : Vpl<G>::value;  // softmax states per lane
   extern __shared__ __align__(128) unsigned char smem[];
   unsigned char* stages = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * kStageBytes);
