@@ -8,6 +8,7 @@ import torch
 
 from oda_cases import (SCALE, Case, assert_attn_close, assert_lse_close)
 from oracle import oda_oracle as O
+import oda_synth
 from sparse_kv_recall_b200 import build as B
 from sparse_kv_recall_b200 import da, oda
 
@@ -105,6 +106,43 @@ def test_local_short_window_cluster_path(G, lens, sink, window):
     pages, _, rows, _ = np.nonzero(c.kbits != old_k)
     slots = {(int(c.bt_h[b, (n - 1) // 16]), (n - 1) % 16) for b, n in enumerate(lens)}
     assert set(zip(pages.tolist(), rows.tolist())) <= slots
+
+
+def _scale_rows_by_position(c, factor_of):
+    """Multiply the K row of every cached position p of every sequence by factor_of(p, n)
+    (n = that sequence's length), in place, and refresh the host copy."""
+    f = torch.ones((c.num_blocks, 16), dtype=torch.float32)
+    bt = c.bt.cpu().numpy()
+    for b, n in enumerate(c.lengths):
+        for p in range(n):
+            f[bt[b, p // 16], p % 16] = factor_of(p, n)
+    c.kc.copy_((c.kc.float() * f.to("cuda")[:, None, :, None]).to(torch.bfloat16))
+    c.snapshot()
+
+
+@pytest.mark.parametrize("G", [1, 2, 4])
+@pytest.mark.parametrize("shape", ["rising", "sharp"])
+def test_extreme_score_ranges(G, shape):
+    """Scores that keep rising along the sequence (K rows scaled by 1 + 8 p / n: the running
+    maximum is raised again and again, by more than any rescale margin) or that are 8x wider
+    than N(0, 1) logits (about 60 base-2 units between a head's largest and typical score):
+    Full and Local against the oracle."""
+    c = Case([300, 2053, 5000], hq=8 * G, hkv=8, seed=300 + G)
+    if shape == "rising":
+        _scale_rows_by_position(c, lambda p, n: 1.0 + 8.0 * p / n)
+    else:
+        c.q.mul_(8.0)
+        c.qbits = oda_synth.bf16_bits(c.q)
+    out, lse = c.out_buffers()
+    _run(c, lambda: oda.oda_decode_full(c.kv, c.q, SCALE, out, c.ws, lse=lse))
+    ref, rlse = c.oracle(lambda b, t: O.full_positions(t))
+    assert_attn_close(out.cpu().numpy(), ref, "full %s G=%d" % (shape, G))
+    assert_lse_close(lse.cpu().numpy(), rlse)
+    out, lse = c.out_buffers()
+    _run(c, lambda: oda.oda_decode_local(c.kv, c.q, 4, 256, SCALE, out, c.ws, lse=lse))
+    ref, rlse = c.oracle(lambda b, t: O.local_positions(t, 4, 256))
+    assert_attn_close(out.cpu().numpy(), ref, "local %s G=%d" % (shape, G))
+    assert_lse_close(lse.cpu().numpy(), rlse)
 
 
 def test_local_equals_full_when_window_covers_history():
