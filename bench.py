@@ -44,7 +44,10 @@ PAGE_BYTES = 2 * 16 * 128 * 2    # K page + V page of one (page, KV head): 8 KB
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0         # B200 HBM3e nominal (~8 TB/s), reported beside the measured peak
 PROFILE = os.path.join(ROOT, "profiles", "decode_full_128k.md")
+LOCAL_PROFILE = os.path.join(ROOT, "profiles", "decode_local_128k.md")
+RECALL_PROFILE = os.path.join(ROOT, "profiles", "recall_h2048.md")
 KERNEL_SOURCES = ["oda_decode.cu", "oda_plan.cuh", "oda_common.cuh"]
+RECALL_SOURCES = ["oda_recall.cu", "oda_recall.cuh", "oda_common.cuh"]
 
 
 def parse_args():
@@ -176,11 +179,12 @@ def measured_peak():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
-    """Hash of the decode kernel's sources with comments and blank lines removed, so that a
-    change of wording does not void the stored ncu counters but any code change does."""
+def kernel_source_hash(sources=None) -> str:
+    """Hash of a kernel's sources (default: the decode kernels') with comments and blank
+    lines removed, so that a change of wording does not void the stored ncu counters but any
+    code change does."""
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in (KERNEL_SOURCES if sources is None else sources):
         text = open(os.path.join(ROOT, "sparse_kv_recall_b200", "csrc", name)).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         text = re.sub(r"//[^\n]*", "", text)
@@ -189,23 +193,44 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(n_ctx_tokens_per_launch: float):
-    """DRAM bytes per Full launch from the committed ncu summary, scaled to this launch's
-    tokens; None when the summary is missing or was taken on other kernel sources."""
-    if not os.path.exists(PROFILE):
-        return None
+def _profile_fields(path: str, sources=None) -> dict:
+    """The machine-readable "- key: value" lines of a committed ncu summary; empty when the
+    summary is missing or was taken on other kernel sources."""
+    if not os.path.exists(path):
+        return {}
     info = {}
-    for line in open(PROFILE):
+    for line in open(path):
         if line.startswith("- ") and ":" in line:
             k, v = line[2:].split(":", 1)
             info[k.strip()] = v.strip().strip("`")
+    return info if info.get("source_sha") == kernel_source_hash(sources) else {}
+
+
+def profiled_traffic(n_ctx_tokens_per_launch: float):
+    """DRAM bytes per Full launch from the committed ncu summary, scaled to this launch's
+    tokens; None when the summary is missing or was taken on other kernel sources."""
+    info = _profile_fields(PROFILE)
     try:
-        if info.get("source_sha") != kernel_source_hash():
-            return None
         per_token = float(info["dram_bytes_per_launch"]) / float(info["tokens_per_launch"])
         return per_token * n_ctx_tokens_per_launch
     except (KeyError, ValueError):
         return None
+
+
+def profiled_step_bytes(layers: int, full_launches_per_step: float, n_ctx_tokens: float):
+    """DRAM bytes one step of the default workload reads and writes, from the committed ncu
+    summaries of its kernels (Local and Full per layer, the recall head once): the
+    "bytes actually read" figure beside the attended (algorithmic) bytes. None when any
+    summary is missing or stale."""
+    try:
+        local = float(_profile_fields(LOCAL_PROFILE)["dram_bytes_per_launch"])
+        recall = float(_profile_fields(RECALL_PROFILE, RECALL_SOURCES)["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+    full = profiled_traffic(n_ctx_tokens)
+    if full is None:
+        return None
+    return layers * local + recall + full_launches_per_step * full
 
 
 # ---------------------------------------------------------------------------------------
@@ -710,6 +735,7 @@ def run_oda(args, dist: Dist):
     dist.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step0 = step
     e0.record(stream)
     for _ in range(K):
         s.feed(step)
@@ -751,6 +777,15 @@ def run_oda(args, dist: Dist):
         "gpu_launches": launches,
         "clocks": clk,
     }
+    if w.name == DEFAULT_WORKLOAD:
+        # DRAM bytes of the step's kernels as ncu counted them (committed summaries), with the
+        # Full launches at the timed region's mean context
+        ctx_mid = float(np.mean(s.lengths)) + step0 + K / 2.0 + 1.0
+        sb = profiled_step_bytes(w.layers, fc[1] * w.layers / float(K), ctx_mid * w.batch)
+        result["kv_stream"]["ncu_bytes_per_step"] = sb
+        result["kv_stream"]["ncu_gbs"] = (sb * K / (ms_local / 1e3) / 1e9) if sb else None
+        result["kv_stream"]["ncu_frac_of_peak"] = (sb * K / (ms_local / 1e3) / 1e9 / peak
+                                                   if sb else None)
     if args.quick:
         return result, s
 

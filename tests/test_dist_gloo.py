@@ -67,3 +67,21 @@ def test_clock_sampler_without_nvidia_smi_is_reported():
     c = bench.ClockSampler(0)
     c.proc = None
     assert c.stop()["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_profiled_bytes_follow_committed_summaries(tmp_path, monkeypatch):
+    """bench.py reads the DRAM bytes of the step's kernels from the committed ncu summaries,
+    and only while the kernel sources they were taken on are unchanged."""
+    import bench
+    full = bench.profiled_traffic(131073)
+    assert full is not None and 1.0 <= full / (131073 * 8 * 512) < 1.05
+    step = bench.profiled_step_bytes(28, 2.0, 131073)
+    local = float(bench._profile_fields(bench.LOCAL_PROFILE)["dram_bytes_per_launch"])
+    recall = float(bench._profile_fields(bench.RECALL_PROFILE,
+                                         bench.RECALL_SOURCES)["dram_bytes_per_launch"])
+    assert step == 28 * local + recall + 2.0 * full
+    stale = tmp_path / "stale.md"
+    stale.write_text(open(bench.LOCAL_PROFILE).read().replace(
+        bench.kernel_source_hash(), "0000000000000000"))
+    monkeypatch.setattr(bench, "LOCAL_PROFILE", str(stale))
+    assert bench.profiled_step_bytes(28, 2.0, 131073) is None
