@@ -179,13 +179,19 @@ def measured_peak():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+HOST_MARK = "// Host side."
+
+
 def kernel_source_hash(sources=None) -> str:
-    """Hash of a kernel's sources (default: the decode kernels') with comments and blank
-    lines removed, so that a change of wording does not void the stored ncu counters but any
-    code change does."""
+    """Hash of a kernel's device code (default: the decode kernels'): each source file up to
+    its "// Host side." section (host argument checks and launch wrappers cannot change what
+    a kernel reads), with comments and blank lines removed, so that a change of wording does
+    not void the stored ncu counters but any change of device code does."""
     h = hashlib.sha256()
     for name in (KERNEL_SOURCES if sources is None else sources):
         text = open(os.path.join(ROOT, "sparse_kv_recall_b200", "csrc", name)).read()
+        if HOST_MARK in text:
+            text = text[:text.index(HOST_MARK)]
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         text = re.sub(r"//[^\n]*", "", text)
         lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]

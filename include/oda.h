@@ -20,6 +20,10 @@
  *     offending work item is skipped; kernels never trap.
  *   - Head dimension 128, page size 16 tokens, bf16 K/V/Q, fp32 accumulation. Query head h
  *     reads KV head h / (num_q_heads / num_kv_heads); the group size must be 1, 2 or 4.
+ *   - Pointer alignment: every device pointer is aligned to its element type (4 bytes for
+ *     int32 and fp32 arrays, 8 for the u64 counters, 2 for bf16 outputs); the K/V caches, q,
+ *     k_new, v_new and every workspace to 16 bytes. A misaligned pointer is rejected with
+ *     ODA_ERR_INVALID_ARG before anything is launched.
  */
 #ifndef ODA_H_
 #define ODA_H_

@@ -48,6 +48,7 @@ extern "C" int oda_kv_append(const oda_kv* kv, const void* k_new, const void* v_
   if (k_new == nullptr || v_new == nullptr) return ODA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15u)
     return ODA_ERR_INVALID_ARG;
+  if (!aligned_or_null(gate, 4)) return ODA_ERR_INVALID_ARG;
   append_kernel<<<kv->batch, 32 * kv->num_kv_heads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<__nv_bfloat16*>(kv->k_cache), static_cast<__nv_bfloat16*>(kv->v_cache),
       kv->block_table, kv->seq_lens, kv->max_blocks_per_seq, kv->num_blocks, kv->num_kv_heads,

@@ -1113,6 +1113,9 @@ int check_kv(const oda_kv* kv) {
                         kv->block_table == nullptr || kv->seq_lens == nullptr))
     return ODA_ERR_INVALID_ARG;
   if (!aligned16(kv->k_cache) || !aligned16(kv->v_cache)) return ODA_ERR_INVALID_ARG;
+  if (!aligned_or_null(kv->block_table, 4) || !aligned_or_null(kv->seq_lens, 4) ||
+      !aligned_or_null(kv->dev_status, 4) || !aligned_or_null(kv->stats, 8))
+    return ODA_ERR_INVALID_ARG;
   return ODA_OK;
 }
 
@@ -1174,6 +1177,10 @@ static bool use_cluster_kernel(const oda_kv* kv, const oda_visibility& vis, cons
 
 int check_visibility(const oda_kv* kv, const oda_visibility* v) {
   if (v == nullptr) return ODA_ERR_INVALID_ARG;
+  if (!aligned_or_null(v->gate, 4) || !aligned_or_null(v->keep_blocks, 4) ||
+      !aligned_or_null(v->keep_counts, 4) || !aligned_or_null(v->da_modes, 4) ||
+      !aligned_or_null(v->da_focus_offsets, 4))
+    return ODA_ERR_INVALID_ARG;
   switch (v->mode) {
     case ODA_MODE_LOCAL:
       return (v->sink < 0 || v->window < 1) ? ODA_ERR_INVALID_ARG : ODA_OK;
@@ -1245,6 +1252,9 @@ int launch_decode(const oda_kv* kv, const oda_visibility& vis, const void* q, in
   if (kv->batch == 0) return ODA_OK;
   if (q == nullptr || out == nullptr || ws == nullptr) return ODA_ERR_INVALID_ARG;
   if (!aligned16(q) || (k_new && (!aligned16(k_new) || !aligned16(v_new))))
+    return ODA_ERR_INVALID_ARG;
+  if (!aligned16(ws) || !aligned_or_null(out, out_dtype == ODA_BF16 ? 2 : 4) ||
+      !aligned_or_null(lse, 4))
     return ODA_ERR_INVALID_ARG;
   DeviceInfo di;
   if ((rc = current_device_info(&di)) != ODA_OK) return rc;

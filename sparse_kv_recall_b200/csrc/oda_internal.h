@@ -11,6 +11,12 @@ namespace oda {
 // Remember the most recent CUDA error seen by this thread (reported by oda_last_cuda_error).
 void note_cuda_error(int err);
 
+// True when p is null or a multiple of `bytes` (a power of two): every pointer a kernel
+// reads or writes as a typed, vector or atomic access is checked on the host with this.
+inline bool aligned_or_null(const void* p, size_t bytes) {
+  return (reinterpret_cast<uintptr_t>(p) & (bytes - 1)) == 0;
+}
+
 // Attribute setup for every decode kernel instantiation on the current device; call before
 // stream capture so that nothing but launches is recorded.
 int prepare_decode_kernels();

@@ -80,6 +80,10 @@ extern "C" int oda_merge_partials(const float* o_parts, const float* lse_parts, 
     return ODA_ERR_UNSUPPORTED_SHAPE;
   if (batch == 0) return ODA_OK;
   if (o_parts == nullptr || lse_parts == nullptr || out == nullptr) return ODA_ERR_INVALID_ARG;
+  if (!aligned_or_null(o_parts, 4) || !aligned_or_null(lse_parts, 4) ||
+      !aligned_or_null(gate, 4) || !aligned_or_null(out, out_dtype == ODA_BF16 ? 2 : 4) ||
+      !aligned_or_null(lse, 4))
+    return ODA_ERR_INVALID_ARG;
   MergeParams p;
   p.o_parts = o_parts;
   p.lse_parts = lse_parts;

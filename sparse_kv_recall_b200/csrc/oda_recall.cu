@@ -187,6 +187,9 @@ __global__ void __maxnreg__(104) recall_kernel(const RecallParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------------------
 int launch_recall(const float* h_prev, const float* emb, const void* h_local, int h_local_dtype,
                   int batch, int hidden, int mlp, const float* w1, const float* b1,
                   const float* w2, float b2, float theta, float* q_out, int32_t* gate_out,
@@ -196,6 +199,14 @@ int launch_recall(const float* h_prev, const float* emb, const void* h_local, in
   if (h_local_dtype != ODA_F32 && h_local_dtype != ODA_BF16) return ODA_ERR_INVALID_ARG;
   if (batch == 0) return ODA_OK;
   if (!h_prev || !emb || !h_local || !w1 || !b1 || !w2 || !q_out || !gate_out || !ws)
+    return ODA_ERR_INVALID_ARG;
+  for (const void* f : {static_cast<const void*>(h_prev), static_cast<const void*>(emb),
+                        static_cast<const void*>(w1), static_cast<const void*>(b1),
+                        static_cast<const void*>(w2), static_cast<const void*>(q_out),
+                        static_cast<const void*>(gate_out)})
+    if (!aligned_or_null(f, 4)) return ODA_ERR_INVALID_ARG;
+  if (!aligned_or_null(h_local, h_local_dtype == ODA_BF16 ? 2 : 4) ||
+      !aligned_or_null(full_count, 8) || !aligned_or_null(ws, 16))
     return ODA_ERR_INVALID_ARG;
   const RecallWs wl = recall_ws(batch, hidden, mlp);
   if (ws_bytes < wl.total) return ODA_ERR_WORKSPACE_TOO_SMALL;

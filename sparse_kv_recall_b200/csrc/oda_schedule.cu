@@ -40,6 +40,8 @@ int launch_gate_schedule(const float* u, int batch, float rho, int32_t* gate_out
   if (batch < 0 || !(rho >= 0.f && rho <= 1.f)) return ODA_ERR_INVALID_ARG;
   if (batch == 0) return ODA_OK;
   if (u == nullptr || gate_out == nullptr) return ODA_ERR_INVALID_ARG;
+  if (!aligned_or_null(u, 4) || !aligned_or_null(gate_out, 4) || !aligned_or_null(full_count, 8))
+    return ODA_ERR_INVALID_ARG;
   gate_schedule_kernel<<<1, kSchedThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       u, batch, rho, gate_out, full_count,
       static_cast<cudaGraphConditionalHandle>(graph_cond_handle), graph_cond_handle != 0ull);

@@ -228,6 +228,15 @@ extern "C" int oda_recall_loss_grad(const float* h_prev, const float* emb, const
   if (!h_prev || !emb || !h_local || !w1 || !b1 || !w2 || !gain || !loss_out || !dw1 || !db1 ||
       !dw2 || !db2 || !ws)
     return ODA_ERR_INVALID_ARG;
+  for (const void* f : {static_cast<const void*>(h_prev), static_cast<const void*>(emb),
+                        static_cast<const void*>(w1), static_cast<const void*>(b1),
+                        static_cast<const void*>(w2), static_cast<const void*>(gain),
+                        static_cast<const void*>(q_out), static_cast<const void*>(loss_out),
+                        static_cast<const void*>(dw1), static_cast<const void*>(db1),
+                        static_cast<const void*>(dw2), static_cast<const void*>(db2)})
+    if (!aligned_or_null(f, 4)) return ODA_ERR_INVALID_ARG;
+  if (!aligned_or_null(h_local, h_local_dtype == ODA_BF16 ? 2 : 4) || !aligned_or_null(ws, 16))
+    return ODA_ERR_INVALID_ARG;
   const TrainWs wl = train_ws(batch, hidden, mlp);
   if (ws_bytes < wl.total) return ODA_ERR_WORKSPACE_TOO_SMALL;
   TrainParams p;

@@ -72,6 +72,15 @@ def test_decode_argument_checks(lib):
     assert _local(lib, _kv(), sink=-1) == I
     assert _local(lib, _kv(), k_new=0x80000) == I         # k_new without v_new
     assert _local(lib, _kv(k_cache=0x10008)) == I         # bulk copies need 16-byte alignment
+    assert _local(lib, _kv(), ws=0x60008) == I             # workspace: 16-byte aligned
+    assert _local(lib, _kv(), out=0x50002) == I            # fp32 output: 4-byte aligned
+    assert _local(lib, _kv(), out=0x50001, out_dtype=1) == I   # bf16 output: 2-byte aligned
+    assert _local(lib, _kv(block_table=0x30002)) == I
+    assert _local(lib, _kv(dev_status=0x90001)) == I
+    assert _local(lib, _kv(stats=0x90004)) == I            # u64 counters: 8-byte aligned
+    kv = _kv()
+    assert lib.oda_decode_full(ctypes.byref(kv), 0x70000, 16, 0.1, 0x80002, None, None, 0x50000,
+                               0, None, 0x60000, 1 << 40, None) == I   # int32 gate: 4-byte
     assert _local(lib, _kv(batch=-1)) == I
     assert _local(lib, _kv(batch=2000)) == U
     assert _local(lib, _kv(batch=0)) == oda.ODA_OK         # nothing to do, nothing launched
@@ -97,10 +106,18 @@ def test_workspace_queries(lib):
         assert lib.oda_recall_workspace_size(b, 2048, 256, ctypes.byref(n)) == oda.ODA_OK
         sizes.append(n.value)
     assert 0 < sizes[0] < sizes[1] < sizes[2]
-    assert lib.oda_recall_score(0x1, 0x2, 0x3, 0, 1, 2048, 96, 0x4, 0x5, 0x6, 0.0, 0.0, 0x7, 0x8,
-                                None, 0, 0x9, 1 << 30, None) == I
-    assert lib.oda_recall_score(0x1, 0x2, 0x3, 0, 1, 2048, 256, 0x4, 0x5, 0x6, 0.0, 0.0, 0x7, 0x8,
-                                None, 0, 0x9, 16, None) == oda.ODA_ERR_WORKSPACE_TOO_SMALL
+    assert lib.oda_recall_score(0x100, 0x200, 0x300, 0, 1, 2048, 96, 0x400, 0x500, 0x600, 0.0,
+                                0.0, 0x700, 0x800, None, 0, 0x900, 1 << 30, None) == I
+    assert lib.oda_recall_score(0x100, 0x200, 0x300, 0, 1, 2048, 256, 0x400, 0x500, 0x600, 0.0,
+                                0.0, 0x700, 0x800, None, 0, 0x900, 16,
+                                None) == oda.ODA_ERR_WORKSPACE_TOO_SMALL
+    # misaligned pointers are refused before any launch: fp32 input, workspace, counters
+    assert lib.oda_recall_score(0x102, 0x200, 0x300, 0, 1, 2048, 256, 0x400, 0x500, 0x600, 0.0,
+                                0.0, 0x700, 0x800, None, 0, 0x900, 1 << 30, None) == I
+    assert lib.oda_recall_score(0x100, 0x200, 0x300, 0, 1, 2048, 256, 0x400, 0x500, 0x600, 0.0,
+                                0.0, 0x700, 0x800, None, 0, 0x908, 1 << 30, None) == I
+    assert lib.oda_recall_score(0x100, 0x200, 0x300, 0, 1, 2048, 256, 0x400, 0x500, 0x600, 0.0,
+                                0.0, 0x700, 0x800, 0xa04, 0, 0x900, 1 << 30, None) == I
 
 
 def test_step_graph_argument_checks(lib):
@@ -158,6 +175,10 @@ def test_merge_and_schedule_argument_checks(lib):
     assert lib.oda_gate_schedule(0x1000, 4, float("nan"), 0x2000, None, 0, None) == I
     assert lib.oda_gate_schedule(None, 4, 0.5, 0x2000, None, 0, None) == I
     assert lib.oda_gate_schedule(0x1000, 0, 0.5, 0x2000, None, 0, None) == OK
+    assert lib.oda_gate_schedule(0x1002, 4, 0.5, 0x2000, None, 0, None) == I
+    assert lib.oda_gate_schedule(0x1000, 4, 0.5, 0x2000, 0x3004, 0, None) == I
+    assert lib.oda_merge_partials(0x1002, 0x2000, 2, 1, 16, None, 0x3000, 0, None, None) == I
+    assert lib.oda_merge_partials(0x1000, 0x2000, 2, 1, 16, None, 0x3001, 1, None, None) == I
 
 
 def test_recall_training_argument_checks(lib):
@@ -169,16 +190,19 @@ def test_recall_training_argument_checks(lib):
     need = n.value
     assert need > 0
 
-    def call(batch=8, mlp=256, delta=1.0, gain=0xa, ws_bytes=None):
-        return lib.oda_recall_loss_grad(0x1, 0x2, 0x3, 0, batch, 2048, mlp, 0x4, 0x5, 0x6, 0.0,
-                                        gain, 0.0, delta, None, 0xb, 0xc, 0xd, 0xe, 0xf, 0x10,
-                                        need if ws_bytes is None else ws_bytes, None)
+    def call(batch=8, mlp=256, delta=1.0, gain=0xa00, ws_bytes=None, ws=0x1000, dw1=0xc00):
+        return lib.oda_recall_loss_grad(0x100, 0x200, 0x300, 0, batch, 2048, mlp, 0x400, 0x500,
+                                        0x600, 0.0, gain, 0.0, delta, None, 0xb00, dw1, 0xd00,
+                                        0xe00, 0xf00, ws, need if ws_bytes is None else ws_bytes,
+                                        None)
     assert call(delta=0.0) == I
     assert call(delta=float("inf")) == I
     assert call(gain=None) == I
     assert call(mlp=96) == I
     assert call(batch=2000) == I
     assert call(ws_bytes=16) == oda.ODA_ERR_WORKSPACE_TOO_SMALL
+    assert call(ws=0x1008) == I                               # workspace: 16-byte aligned
+    assert call(dw1=0xc02) == I                               # fp32 output: 4-byte aligned
     assert call(batch=0) == oda.ODA_OK
 
 
