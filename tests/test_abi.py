@@ -91,6 +91,8 @@ def test_decode_argument_checks(lib):
                                     0, None, 0x60000, 1, None) == I   # max_keep > pages per seq
     assert lib.oda_kv_append(ctypes.byref(_kv(num_kv_heads=40)), 0x1000, 0x2000, None, None) == U
     assert lib.oda_kv_append(ctypes.byref(_kv()), None, 0x2000, None, None) == I
+    assert lib.oda_kv_append(ctypes.byref(_kv()), 0x1000, 0x2008, None, None) == I   # 16 bytes
+    assert lib.oda_kv_append(ctypes.byref(_kv()), 0x1000, 0x2000, 0x3002, None) == I  # gate
     assert lib.oda_visible_mask(ctypes.byref(_kv()), 9, 4, 256, None, None, None, 0, 0x1000, 10,
                                 None) == I
 
