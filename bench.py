@@ -43,11 +43,12 @@ ROW_BYTES = 2 * 128 * 2          # K row + V row of one (position, KV head): 512
 PAGE_BYTES = 2 * 16 * 128 * 2    # K page + V page of one (page, KV head): 8 KB
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0         # B200 HBM3e nominal (~8 TB/s), reported beside the measured peak
-PROFILE = os.path.join(ROOT, "profiles", "decode_full_128k.md")
-LOCAL_PROFILE = os.path.join(ROOT, "profiles", "decode_local_128k.md")
-RECALL_PROFILE = os.path.join(ROOT, "profiles", "recall_h2048.md")
-KERNEL_SOURCES = ["oda_decode.cu", "oda_plan.cuh", "oda_common.cuh"]
-RECALL_SOURCES = ["oda_recall.cu", "oda_recall.cuh", "oda_common.cuh"]
+# Machine-readable ncu figures (written by `bench.py --ncu-summary` from a capture's raw CSV),
+# beside the prose summaries of the same captures in profiles/*.md.
+PROFILE = os.path.join(ROOT, "profiles", "full_chain_128k.json")
+LOCAL_PROFILE = os.path.join(ROOT, "profiles", "local_chain_128k.json")
+KERNEL_SOURCES = ["oda_decode.cuh", "oda_decode.cu", "oda_chain.cu", "oda_plan.cuh",
+                  "oda_common.cuh", "oda_recall.cuh"]
 
 
 def parse_args():
@@ -66,12 +67,18 @@ def parse_args():
                     help="skip the 4K-history gate-overhead point")
     ap.add_argument("--no-da", action="store_true",
                     help="skip the block-mask (Declarative Attention) sub-measurement")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the short runs of the other workloads")
     ap.add_argument("--quick", action="store_true",
                     help="main timed region only (used for profiler launch lists)")
-    ap.add_argument("--no-conditional", action="store_true",
-                    help="Full kernels launch every step and skip ungated sequences on-device "
-                         "instead of sitting behind a graph IF node (ncu can list kernel nodes "
-                         "only of graphs without conditional nodes)")
+    ap.add_argument("--conditional", action="store_true",
+                    help="put the Full phase behind a graph IF node set by the gate, instead of "
+                         "the default device-side early exit of the persistent Full kernel (ncu "
+                         "lists kernel nodes only of graphs without conditional nodes)")
+    ap.add_argument("--step-kernels", choices=["persistent", "per-layer"], default="persistent",
+                    help="persistent: Local at every layer with the fused gate, and Full at "
+                         "every layer, as one launch each; per-layer: one launch per layer "
+                         "and phase")
     ap.add_argument("--profile-kernel", choices=["full", "local", "recall", "train"],
                     help="one layer of the workload, the named kernel launched --steps times "
                          "(a small case for ncu captures); prints nothing")
@@ -200,43 +207,87 @@ def kernel_source_hash(sources=None) -> str:
 
 
 def _profile_fields(path: str, sources=None) -> dict:
-    """The machine-readable "- key: value" lines of a committed ncu summary; empty when the
-    summary is missing or was taken on other kernel sources."""
+    """The figures of a committed ncu capture (a JSON file written by --ncu-summary); empty when
+    the file is missing or was taken on other kernel sources."""
     if not os.path.exists(path):
         return {}
-    info = {}
-    for line in open(path):
-        if line.startswith("- ") and ":" in line:
-            k, v = line[2:].split(":", 1)
-            info[k.strip()] = v.strip().strip("`")
+    try:
+        info = json.load(open(path))
+    except ValueError:
+        return {}
     return info if info.get("source_sha") == kernel_source_hash(sources) else {}
 
 
-def profiled_traffic(n_ctx_tokens_per_launch: float):
-    """DRAM bytes per Full launch from the committed ncu summary, scaled to this launch's
-    tokens; None when the summary is missing or was taken on other kernel sources."""
+def profiled_traffic(n_ctx_tokens_per_layer: float, layers: int = 1):
+    """DRAM bytes of a Full launch covering `layers` layers at this many context tokens per
+    layer, from the committed ncu capture of the persistent Full kernel (scaled by tokens and
+    layers, as its traffic grows in proportion); None when missing or stale."""
     info = _profile_fields(PROFILE)
     try:
-        per_token = float(info["dram_bytes_per_launch"]) / float(info["tokens_per_launch"])
-        return per_token * n_ctx_tokens_per_launch
-    except (KeyError, ValueError):
+        per_token = float(info["dram_bytes_per_launch"]) / (
+            float(info["tokens_per_layer"]) * float(info["layers_per_launch"]))
+        return per_token * n_ctx_tokens_per_layer * layers
+    except (KeyError, ValueError, ZeroDivisionError):
         return None
 
 
-def profiled_step_bytes(layers: int, full_launches_per_step: float, n_ctx_tokens: float):
+def profiled_step_bytes(layers: int, full_phases_per_step: float, n_ctx_tokens: float):
     """DRAM bytes one step of the default workload reads and writes, from the committed ncu
-    summaries of its kernels (Local and Full per layer, the recall head once): the
-    "bytes actually read" figure beside the attended (algorithmic) bytes. None when any
-    summary is missing or stale."""
+    captures of its kernels (the persistent Local kernel with the fused recall head, the
+    persistent Full kernel on the steps that run it): the "bytes actually read" figure beside
+    the attended (algorithmic) bytes. None when any capture is missing or stale."""
     try:
-        local = float(_profile_fields(LOCAL_PROFILE)["dram_bytes_per_launch"])
-        recall = float(_profile_fields(RECALL_PROFILE, RECALL_SOURCES)["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
+        loc = _profile_fields(LOCAL_PROFILE)
+        local = float(loc["dram_bytes_per_launch"]) * layers / float(loc["layers_per_launch"])
+    except (KeyError, ValueError, ZeroDivisionError):
         return None
-    full = profiled_traffic(n_ctx_tokens)
+    full = profiled_traffic(n_ctx_tokens, layers)
     if full is None:
         return None
-    return layers * local + recall + full_launches_per_step * full
+    return local + full_phases_per_step * full
+
+
+def ncu_summary(csv_path: str, kernel: str, out_path: str, extra: dict) -> dict:
+    """Average per-launch DRAM bytes of the launches of `kernel` (a substring of the kernel
+    name) in an `ncu --page raw --csv` export, written as JSON with the hash of the device
+    sources they were taken on and the caller's description of the launch (`extra`)."""
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    head = None
+    for i, r in enumerate(rows):
+        if "Kernel Name" in r:
+            head, rows = r, rows[i + 1:]
+            break
+    if head is None:
+        raise ValueError("no header row in %s" % csv_path)
+    ki = head.index("Kernel Name")
+    cols = {m: head.index(m) for m in ("dram__bytes_read.sum", "dram__bytes_write.sum",
+                                       "gpu__time_duration.sum") if m in head}
+    units = rows[0] if rows and not rows[0][ki] else None
+    scale = {}
+    for m, j in cols.items():
+        u = (units[j] if units else "").strip().lower()
+        scale[m] = {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "ns": 1e-9, "us": 1e-6,
+                    "usecond": 1e-6, "msecond": 1e-3, "nsecond": 1e-9}.get(u, 1)
+    picked = [r for r in rows if len(r) > ki and kernel in r[ki]]
+    if not picked:
+        raise ValueError("no launch of %s in %s" % (kernel, csv_path))
+
+    def mean(m):
+        vals = [float(r[cols[m]].replace(",", "")) * scale[m] for r in picked]
+        return sum(vals) / len(vals)
+
+    info = dict(extra)
+    info.update({"kernel": picked[0][ki][:120], "launches_captured": len(picked),
+                 "source_sha": kernel_source_hash(),
+                 "dram_bytes_read_per_launch": mean("dram__bytes_read.sum"),
+                 "dram_bytes_write_per_launch": mean("dram__bytes_write.sum")})
+    info["dram_bytes_per_launch"] = (info["dram_bytes_read_per_launch"]
+                                     + info["dram_bytes_write_per_launch"])
+    if "gpu__time_duration.sum" in cols:
+        info["gpu_time_s_per_launch_under_ncu"] = mean("gpu__time_duration.sum")
+    json.dump(info, open(out_path, "w"), indent=1)
+    return info
 
 
 # ---------------------------------------------------------------------------------------
@@ -246,7 +297,7 @@ class Setup:
     """Caches, recall head, engine and the resident pool of per-step inputs."""
 
     def __init__(self, w, seed_offset: int, n_steps_total: int, theta: float, dev: str,
-                 use_conditional: bool = True):
+                 use_conditional: bool = False, step_kernels: int = 0):
         from sparse_kv_recall_b200.engine import OdaEngine, StagingLayout, fill_staging
         self.w = oda_synth.scaled(w, seed=w.seed + 1000 * seed_offset)
         w = self.w
@@ -260,7 +311,8 @@ class Setup:
         self.recall = (rw.w1, rw.b1, rw.w2, rw.b2)
         self.eng = OdaEngine([c[0] for c in self.caches], [c[1] for c in self.caches],
                              self.layout.block_table, w.num_q_heads, self.recall, theta,
-                             sink=w.sink, window=w.window, use_conditional=use_conditional)
+                             sink=w.sink, window=w.window, use_conditional=use_conditional,
+                             step_kernels=step_kernels)
         self.eng.set_h_prev(oda_synth.make_h0(w, device=dev), 0)
         lay = StagingLayout(w.layers, w.batch, w.num_q_heads, w.num_kv_heads, w.hidden)
         self.slot = lay.nbytes
@@ -274,9 +326,11 @@ class Setup:
         self.eng.staging.copy_(self.pool[i], non_blocking=True)
 
 
-def launches_per_step(w, phases: int, steps: int, conditional: bool = True) -> int:
-    """Kernels of this library launched by `steps` steps of which `phases` ran Full."""
-    return steps * (w.layers + 1) + (phases if conditional else steps) * w.layers
+def launches_per_step(kernels, phases: int, steps: int, conditional: bool = True) -> int:
+    """Kernels of this library launched by `steps` steps of which `phases` ran Full, for a
+    step graph launching kernels = (Local, gate, Full) kernels per step."""
+    local, gate, full = kernels
+    return steps * (local + gate) + (phases if conditional else steps) * full
 
 
 def calibrate_theta(s, w, C: int, step: int):
@@ -338,22 +392,44 @@ def phase_breakdown(s, w, theta: float, PH: int, step: int, stream):
     mean = lambda xs: float(np.mean(xs)) if xs else None
     T_step, T_loc = mean(t_step), mean(t_local)
     T_full_exec = sum(t_full[i] for i in full_steps) / PH if PH else 0.0
-    gate_over = (T_step - T_loc - T_full_exec) / T_step if T_step else None
+    # The Local kernels alone (the same graphs captured with the Local phase only, event nodes
+    # around it): with the persistent kernels the gate runs inside the Local launch, so the
+    # step's Local phase above includes it and only this measurement separates them.
+    from sparse_kv_recall_b200 import oda
+    lo = eng.capture(math.inf, oda.ODA_PHASE_LOCAL)
+    t_lo = []
+    for i in range(min(PH, 64)):
+        lo[step % 2].set_events(*evs[i])
+        s.feed(step)
+        lo[step % 2].launch()
+        step += 1
+        if i % 16 == 15:
+            torch.cuda.synchronize()
+            t_lo += [evs[k][0].elapsed_time(evs[k][1]) for k in range(i - 15, i + 1)]
+    torch.cuda.synchronize()
+    for x in lo:
+        x.close()
+    T_lo = mean(t_lo)
+    gate_over = (T_step - T_lo - T_full_exec) / T_step if T_step and T_lo else None
     local_rows = sum(min(n + step - PH / 2 + 1, w.sink + w.window) for n in s.lengths)
     eng.timing = False
     eng.set_theta(theta)
     return {
         "steps": PH, "steps_with_full": len(full_steps), "ms_step": T_step, "ms_local_phase": T_loc,
+        "ms_local_kernels_alone": T_lo,
         "ms_recall": mean(t_recall), "ms_full_phase_when_run": mean([t_full[i] for i in full_steps]),
         "ms_full_phase_when_skipped": mean([t_full[i] for i in local_steps]),
         "gate_overhead": gate_over,
-        "gate_overhead_def": "(step - Local phase - executed Full phase) / step; recall and IF "
-                             "node timed without PDL between event nodes",
+        "gate_overhead_def": "(T_step - T_local - T_full_executed) / T_step with event nodes at the "
+                             "phase boundaries: T_step and the executed Full phase (summed over the "
+                             "steps that ran it, divided by all steps) from the step graphs, T_local "
+                             "from the Local-only graph (the gate excluded)",
         "local_phase_kv_gbs": (w.layers * w.num_kv_heads * local_rows * ROW_BYTES
-                               / (T_loc / 1e3) / 1e9) if T_loc else None,
+                               / (T_lo / 1e3) / 1e9) if T_lo else None,
         "full_phase_kv_gbs": (sum(full_bytes[i] for i in full_steps)
                               / (sum(t_full[i] for i in full_steps) / 1e3) / 1e9)
                              if full_steps else None,
+        "full_bytes_per_phase": mean([full_bytes[i] for i in full_steps]),
     }, step
 
 
@@ -412,17 +488,22 @@ def gate_cost(s, w, theta: float, n: int, step: int, stream, rounds: int = 4):
             x.close()
     T = {name: float(np.median(v)) for name, v in times.items()}
     overhead = T["theta_plus_inf"] - T["local_only"]
+    rho = gated / float(w.batch * n * rounds)
+    full = T["theta_minus_inf"] - T["theta_plus_inf"]
     return {"ms_per_step": T, "rounds": rounds, "steps_per_round": n,
-            "rho_realised": gated / float(w.batch * n * rounds),
-            "ms_recall_and_if_node": overhead,
-            "ms_recall_head": T["local_recall"] - T["local_only"],
-            "ms_if_node_skipped": T["theta_plus_inf"] - T["local_recall"],
-            "ms_full_phase": T["theta_minus_inf"] - T["theta_plus_inf"],
+            "rho_realised": rho,
+            "ms_gate_and_full_skip": overhead,
+            "ms_gate": T["local_recall"] - T["local_only"],
+            "ms_full_phase_skipped": T["theta_plus_inf"] - T["local_recall"],
+            "ms_full_phase": full,
             "gate_overhead": overhead / T["oda"],
             "gate_overhead_def": "(T(theta=+inf) - T(Local-only graph)) / T(calibrated theta): "
-                                 "recall head + IF node per step over the whole step, same "
-                                 "PDL-chained graphs, no event nodes inside, medians of "
-                                 "interleaved rounds"}, step
+                                 "the gate and the skipped Full phase per step over the whole "
+                                 "step, graphs without event nodes, medians of interleaved rounds",
+            "gate_overhead_survey": (T["oda"] - T["local_only"] - rho * full) / T["oda"],
+            "gate_overhead_survey_def": "(T_step - T_local - T_full_executed) / T_step from the same "
+                                        "graphs without event nodes: T_full_executed = realised rho "
+                                        "x (T(theta=-inf) - T(theta=+inf))"}, step
 
 
 def step_variants(s, w, theta: float, rho: float, n: int, step: int, stream):
@@ -538,12 +619,52 @@ def run_train_grad(w, dev, stream, batch: int = 8, reps: int = 50):
             "gbs": nbytes / (us / 1e6) / 1e9, "loss": float(loss.item())}
 
 
+def run_brief(name: str, dev: str, stream, steps: int = 64, with_gate_cost: bool = False):
+    """A short run of another workload through the same step graphs: theta calibrated to its
+    target Full-call rate (or its fixed theta), `steps` timed steps; tokens/s, the realised
+    rate and the KV bytes it attended per second."""
+    w = oda_synth.WORKLOADS[name]
+    C = 0 if w.theta is not None else 256
+    GC = 16 if with_gate_cost else 0
+    total = C + 8 + steps + (5 * 4 * (GC + 4) if GC else 0) + 8
+    s = Setup(w, 0, total, float("inf") if w.theta is None else w.theta, dev)
+    theta, step = w.theta, 0
+    if theta is None:
+        theta, step = calibrate_theta(s, w, C, step)
+        s.eng.set_theta(theta)
+    for _ in range(8):
+        s.feed(step)
+        s.eng.launch(step)
+        step += 1
+    torch.cuda.synchronize()
+    fc0, st0 = s.eng.full_count.clone(), s.eng.stats.clone()
+    ms, step = timed_steps(s, steps, step, stream)
+    fc = (s.eng.full_count - fc0).cpu().tolist()
+    st = (s.eng.stats - st0).cpu().tolist()
+    peak, peak_kind = measured_peak()
+    kv = st[0] * ROW_BYTES / (ms * steps / 1e3) / 1e9
+    res = {"workload": w.name, "layers": w.layers, "batch": w.batch, "q_heads": w.num_q_heads,
+           "kv_heads": w.num_kv_heads, "prefill": w.prefill if w.ragged is None else
+           "U%s" % (list(w.ragged),), "steps": steps, "ms_per_step": ms,
+           "tokens_per_s": w.batch / (ms / 1e3), "rho_target": w.target_rho, "theta": theta,
+           "rho_realised": fc[0] / float(w.batch * steps), "kv_gbs": kv,
+           "frac_of_peak": kv / peak, "peak_kind": peak_kind,
+           "kernels_per_step": s.eng.graphs[0].kernels()}
+    if GC:
+        res["gate_cost"], step = gate_cost(s, w, theta, GC, step, stream)
+    assert int(s.eng.status.item()) == 0
+    s.eng.close()
+    del s
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_gate_point(args, dev, stream, prefill: int = 4096, steps: int = 256):
     """The gate-overhead point: the default workload's shapes with a short history."""
     w = oda_synth.scaled(oda_synth.WORKLOADS[args.workload], prefill=prefill,
                          name=args.workload + "@%d" % prefill)
     C, W = 256, 8
-    s = Setup(w, 0, C + W + 5 * 4 * (steps // 4 + 4) + steps + 64, float("inf"), dev)
+    s = Setup(w, 0, C + W + 5 * 4 * (steps // 4 + 4) + steps + 128, float("inf"), dev)
     theta, step = calibrate_theta(s, w, C, 0)
     s.eng.set_theta(theta)
     for _ in range(W):
@@ -713,9 +834,12 @@ def run_oda(args, dist: Dist):
     GC = 0 if args.quick else 64
     E2E = 0 if (args.quick or args.no_e2e) else min(K, 256)
     VAR = 0 if args.quick else 128
-    total = C + W + K + PH + (5 * 4 * (GC + 4) if GC else 0) + E2E + (2 * VAR + 16 if VAR else 0)
+    total = (C + W + K + PH + min(PH, 64) + (5 * 4 * (GC + 4) if GC else 0) + E2E
+             + (2 * VAR + 16 if VAR else 0))
     s = Setup(w, dist.rank, total, float("inf") if w.theta is None else w.theta, dev,
-              use_conditional=not args.no_conditional)
+              use_conditional=args.conditional,
+              step_kernels=oda.ODA_STEP_PER_LAYER if args.step_kernels == "per-layer"
+              else oda.ODA_STEP_PERSISTENT)
     eng = s.eng
     stream = torch.cuda.current_stream()
     step = 0
@@ -760,7 +884,8 @@ def run_oda(args, dist: Dist):
     rho = fc[0] / float(w.batch * K)
     kv_bytes = st[0] * ROW_BYTES
     page_bytes = st[1] * PAGE_BYTES
-    launches = launches_per_step(w, fc[1], K, not args.no_conditional)
+    kernels = eng.graphs[0].kernels()
+    launches = launches_per_step(kernels, fc[1], K, args.conditional)
     peak, peak_kind = measured_peak()
     result = {
         "metric": METRIC, "value": tokens / (ms / 1e3), "unit": UNIT, "n_gpus": dist.world,
@@ -771,8 +896,8 @@ def run_oda(args, dist: Dist):
                    "kv_heads": w.num_kv_heads, "head_dim": 128, "prefill": w.prefill,
                    "sink": w.sink, "window": w.window, "kv_dtype": "bf16",
                    "rho_target": w.target_rho, "rho_realised": rho, "theta": theta,
-                   "calibration_steps": C, "full_phase": "device early exit (no IF node)"
-                   if args.no_conditional else "graph IF node", "l2": "no flush: 15 GB KV stream per Full step >> 126 MB L2"
+                   "calibration_steps": C, "full_phase": "graph IF node" if args.conditional
+                   else "device early exit (no IF node)", "l2": "no flush: 15 GB KV stream per Full step >> 126 MB L2"
                    if w.name == DEFAULT_WORKLOAD else "no flush: KV working set > L2",
                    "parallelism": "replicas (dp%d, no collective)" % dist.world},
         "kv_stream": {"attended_bytes": kv_bytes, "gbs": kv_bytes / (ms_local / 1e3) / 1e9,
@@ -780,14 +905,18 @@ def run_oda(args, dist: Dist):
                       "page_bytes": page_bytes, "peak_gbs": peak, "peak_kind": peak_kind,
                       "frac_of_nominal": kv_bytes / (ms_local / 1e3) / 1e9 / NOMINAL_HBM_GBS,
                       "nominal_gbs": NOMINAL_HBM_GBS},
+        "rho_realised": rho,
+        "hbm_frac_whole_step": kv_bytes / (ms_local / 1e3) / 1e9 / peak,
         "gpu_launches": launches,
+        "kernels_per_step": {"local": kernels[0], "gate": kernels[1], "full": kernels[2],
+                             "step_kernels": args.step_kernels},
         "clocks": clk,
     }
     if w.name == DEFAULT_WORKLOAD:
         # DRAM bytes of the step's kernels as ncu counted them (committed summaries), with the
         # Full launches at the timed region's mean context
         ctx_mid = float(np.mean(s.lengths)) + step0 + K / 2.0 + 1.0
-        sb = profiled_step_bytes(w.layers, fc[1] * w.layers / float(K), ctx_mid * w.batch)
+        sb = profiled_step_bytes(w.layers, fc[1] / float(K), ctx_mid * w.batch)
         result["kv_stream"]["ncu_bytes_per_step"] = sb
         result["kv_stream"]["ncu_gbs"] = (sb * K / (ms_local / 1e3) / 1e9) if sb else None
         result["kv_stream"]["ncu_frac_of_peak"] = (sb * K / (ms_local / 1e3) / 1e9 / peak
@@ -808,9 +937,21 @@ def run_oda(args, dist: Dist):
         result[name] = {"tokens_per_s": w.batch / (T[key] / 1e3), "ms_per_step": T[key],
                         "kv_gbs": kv / (T[key] / 1e3) / 1e9,
                         "frac_of_peak": kv / (T[key] / 1e3) / 1e9 / peak}
+    # the same step at the target Full-call rate, from the interleaved timings: the step without
+    # Full plus the target share of the Full phase (a step's time is linear in its Full calls)
+    gc = result["gate_cost"]
+    if w.target_rho is not None:
+        ms_t = T["theta_plus_inf"] + w.target_rho * gc["ms_full_phase"]
+        kv_t = w.batch * w.layers * w.num_kv_heads * ROW_BYTES * (
+            min(ctx, w.sink + w.window) + w.target_rho * ctx)
+        result["at_target_rho"] = {
+            "rho": w.target_rho, "ms_per_step": ms_t, "tokens_per_s": w.batch / (ms_t / 1e3),
+            "kv_gbs": kv_t / (ms_t / 1e3) / 1e9, "frac_of_peak": kv_t / (ms_t / 1e3) / 1e9 / peak,
+            "how": "T(theta=+inf) + rho x (T(theta=-inf) - T(theta=+inf)) from gate_cost's "
+                   "interleaved medians; KV bytes at the same context"}
     result["variants"], step = step_variants(s, w, theta, rho, VAR, step, stream)
 
-    # ---- dominant kernel alone: Full decode at this context, CUDA events per launch ----
+    # ---- one Full layer alone: the split decode kernel at this context, CUDA events per launch
     from sparse_kv_recall_b200 import oda as O
     ones = torch.ones(w.batch, dtype=torch.int32, device=dev)
     out = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float32, device=dev)
@@ -827,25 +968,35 @@ def run_oda(args, dist: Dist):
     torch.cuda.synchronize()
     dur = float(np.mean([a.elapsed_time(b) for a, b in kevs]))
     ctx_tokens = int(eng.seq_lens.sum().item())
-    alg = ctx_tokens * w.num_kv_heads * ROW_BYTES
-    achieved_alone = alg / (dur / 1e3) / 1e9
-    traffic = profiled_traffic(ctx_tokens)
-    # The dominant kernel as the step runs it: the Full phase (w.layers launches chained with
-    # programmatic dependent launch) timed by event nodes at its boundaries, per launch; its
-    # bytes per launch at that phase's context. Alone: one launch between two events.
+    alg_layer = ctx_tokens * w.num_kv_heads * ROW_BYTES
+    achieved_alone = alg_layer / (dur / 1e3) / 1e9
+    # The dominant kernel as the step runs it: the Full phase -- one persistent launch over
+    # every layer (or one launch per layer, chained by programmatic dependent launch) -- timed
+    # by event nodes at its boundaries on the graph's stream; its bytes are the gated
+    # sequences' histories at every layer at the phase's context.
     ph = result["phases"]
+    full_launches = kernels[2]
     if ph.get("full_phase_kv_gbs"):
-        achieved, how = ph["full_phase_kv_gbs"], ("Full phase inside the step graph (%d launches "
-                                                  "between event nodes, PDL-chained)" % w.layers)
-        ms_launch = ph["ms_full_phase_when_run"] / w.layers
+        achieved = ph["full_phase_kv_gbs"]
+        alg = ph["full_bytes_per_phase"] / full_launches
+        ms_launch = ph["ms_full_phase_when_run"] / full_launches
+        how = ("the Full phase inside the step graph between event nodes: %d launch%s per step"
+               % (full_launches, "" if full_launches == 1 else "es, PDL-chained"))
     else:
-        achieved, how, ms_launch = achieved_alone, "one launch between two events", dur
-    result["roofline"] = {"kernel": "oda_decode_full (decode_kernel<%d>)" % w.group,
+        achieved, alg, ms_launch, how = achieved_alone, alg_layer, dur, "one layer alone"
+    traffic = profiled_traffic(alg / (w.num_kv_heads * ROW_BYTES * w.layers), w.layers) \
+        if full_launches == 1 else profiled_traffic(alg / (w.num_kv_heads * ROW_BYTES), 1)
+    name = ("full_chain_kernel<%d> (Full at every layer, one launch)" % w.group
+            if full_launches == 1 else "decode_kernel<%d> (Full, one layer)" % w.group)
+    result["roofline"] = {"kernel": name,
                           "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                           "frac": achieved / peak, "traffic": traffic,
                           "algorithmic_bytes": alg, "ms_per_launch": ms_launch, "timed": how,
-                          "achieved_alone": achieved_alone, "frac_alone": achieved_alone / peak,
-                          "ms_per_launch_alone": dur, "peak_kind": peak_kind + " (copy)",
+                          "one_layer_alone": {"kernel": "decode_kernel<%d>" % w.group,
+                                              "achieved": achieved_alone,
+                                              "frac": achieved_alone / peak, "ms": dur,
+                                              "algorithmic_bytes": alg_layer},
+                          "peak_kind": peak_kind + " (copy)",
                           "frac_of_nominal": achieved / NOMINAL_HBM_GBS}
 
     if w.name == DEFAULT_WORKLOAD:
@@ -887,6 +1038,27 @@ def run_oda(args, dist: Dist):
                                            stream, e2e=False)
         result["da_device_modes_1m"] = run_da(oda_synth.WORKLOADS["da-1m-b2"], dist, 128, 4, dev,
                                               stream, e2e=False, device_modes=True)
+    if not args.no_workloads and w.name == DEFAULT_WORKLOAD:
+        # every other workload, briefly, through the same step graphs (this one's buffers freed
+        # first: the ragged batch alone holds 87 GB of KV)
+        s.eng.close()
+        del s, eng
+        torch.cuda.empty_cache()
+        s = None
+        wl = {}
+        wl["pr1-ref-4k"] = run_brief("pr1-ref-4k", dev, stream, steps=64, with_gate_cost=True)
+        for name in ("qwen3-1.7b-16k-b8", "qwen3-8b-ragged-b16"):
+            wl[name] = run_brief(name, dev, stream, steps=64)
+        wl[w.name] = {"workload": w.name, "see": "the main line", "tokens_per_s": result["value"],
+                      "rho_realised": rho, "kv_gbs": result["kv_stream"]["gbs"],
+                      "frac_of_peak": result["kv_stream"]["frac_of_peak"]}
+        if "da_device_modes_1m" in result:
+            d = result["da_device_modes_1m"]
+            wl["da-1m-b2"] = {"workload": "da-1m-b2", "tokens_per_s": d["tokens_per_s"],
+                              "rho_realised": None, "kv_gbs": d["kv_gbs"],
+                              "frac_of_peak": d["kv_gbs"] / peak,
+                              "note": "block-mask mode: no gate (device-compiled DA modes)"}
+        result["workloads"] = wl
     return result, s
 
 
@@ -925,8 +1097,10 @@ class OracleSampler:
         self.rec = [x.double().numpy() for x in (rw.w1, rw.b1, rw.w2)] + [rw.b2]
         self.h = np.random.default_rng(0).standard_normal((3, w.batch, w.hidden))
 
-    def sample(self, i: int) -> float:
-        """Seconds of one extrapolated oracle decode step (per sequence of the batch)."""
+    def sample(self, i: int):
+        """One bounded sample: (seconds it took, seconds a whole decode step of the batch
+        would take at the same rates, i.e. the sample's time scaled by the share of the step's
+        attended rows and recall work it covers)."""
         O, w = self.O, self.w
         G = w.num_q_heads // w.num_kv_heads
         qf = O.widen_bf16(self.qbits)
@@ -946,26 +1120,84 @@ class OracleSampler:
         t3 = time.perf_counter()
         per_seq = (w.layers * (t1 - t0)
                    + self.rho * w.layers * w.num_kv_heads * self.chunks * (t3 - t2))
-        return w.batch * per_seq + (t2 - t1)
+        return t3 - t0, w.batch * per_seq + (t2 - t1)
+
+
+def host_cores() -> dict:
+    return {"host_cores": os.cpu_count(), "blas_threads": _blas_threads()}
 
 
 def cpu_baseline(w, rho: float, dev: str, budget_s: float = 20.0) -> dict:
+    """The oracle on the host at the bench's workload: bounded samples, extrapolated."""
     s = OracleSampler(w, rho, dev)
     spent, n, total = 0.0, 0, 0.0
     while spent < budget_s and n < 64:
-        a = time.perf_counter()
-        total += s.sample(n)
-        spent += time.perf_counter() - a
+        wall, whole = s.sample(n)
+        total += whole
+        spent += wall
         n += 1
-    return {"value": w.batch * n / total, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": ("%d oracle samples of one %s decode step (Local at one layer, recall, Full "
-                       "at one layer for one KV head), extrapolated to all %d layers, %d KV heads "
-                       "and rho=%.3f; %.1f s of CPU time" % (n, w.name, w.layers, w.num_kv_heads,
-                                                             rho, spent))}
+    res = {"value": w.batch * n / total, "unit": UNIT, "cores": _blas_threads(),
+           "kind": "oracle", "extrapolated": True,
+           "sample": ("%d oracle samples of one %s decode step (Local at one layer, recall, Full "
+                      "at one layer for one KV head), EXTRAPOLATED by their share of the step's "
+                      "work to all %d layers, %d KV heads and rho=%.3f; %.1f s of CPU time"
+                      % (n, w.name, w.layers, w.num_kv_heads, rho, spent))}
+    res.update(host_cores())
+    return res
+
+
+def cpu_baseline_full(name: str = "pr1-ref-4k") -> dict:
+    """The oracle on the host over a whole small workload, every step, no extrapolation: the
+    1-layer 4K workload (batch 1, 16 q / 8 KV heads, s = 4, w = 256, theta = 0, 64 steps), its
+    inputs drawn on the host by the same seeded generators."""
+    from oracle import oda_oracle as O
+    w = oda_synth.WORKLOADS[name]
+    lengths = oda_synth.prefill_lengths(w)
+    lay = oda_synth.make_layout(w, extra_tokens=w.steps + 2, device="cpu")
+    bt = lay.block_table.numpy()
+    hist = []
+    for l in range(w.layers):
+        pair = []
+        for t in oda_synth.make_kv_cache(w, lay, l, device="cpu"):
+            bits = oda_synth.bf16_bits(t)
+            arr = np.zeros((w.batch, w.num_kv_heads, max(lay.capacity), 128), dtype=np.uint16)
+            for b, cap in enumerate(lay.capacity):
+                p = np.arange(cap)
+                arr[b, :, :cap] = bits[bt[b, p // 16], :, p % 16, :].transpose(1, 0, 2)
+            pair.append(arr)
+        hist.append(pair)
+    rw = oda_synth.make_recall_weights(w)
+    rec = (rw.w1.double().numpy(), rw.b1.double().numpy(), rw.w2.double().numpy(), rw.b2)
+    dec = O.OdaDecoder([h[0] for h in hist], [h[1] for h in hist], lengths,
+                       oda_synth.make_h0(w).double().numpy(), rec, sink=w.sink,
+                       window=w.window, theta=w.theta)
+    inputs = []
+    for i in range(w.steps):
+        si = oda_synth.make_step_inputs(w, i)
+        inp = {k: [oda_synth.bf16_bits(x) for x in getattr(si, k)]
+               for k in ("q_local", "k_local", "v_local", "q_full", "k_full", "v_full")}
+        inp["emb"] = si.emb.double().numpy()
+        inputs.append(inp)
+    gated = 0
+    t0 = time.perf_counter()
+    for inp in inputs:
+        _, _, _, g = dec.step(inp)
+        gated += int(np.sum(g))
+    wall = time.perf_counter() - t0
+    res = {"workload": w.name, "value": w.batch * w.steps / wall, "unit": UNIT, "kind": "oracle",
+           "extrapolated": False, "steps": w.steps, "seconds": wall,
+           "rho_realised": gated / float(w.batch * w.steps),
+           "sample": "every step of the workload through the oracle's ODA step (Local, recall "
+                     "head, gate, Full when gated, commit), timed as one region"}
+    res.update(host_cores())
+    res["cores"] = res["blas_threads"]
+    return res
 
 
 def run_reference(args, dist: Dist):
-    """The oracle, as it stands, timed on the host cores on this workload."""
+    """The oracle, as it stands, timed on the host cores on this workload. Each step is one
+    bounded sample of a decode step; the line's ms_per_step is the real wall time of a sample
+    and its tokens/s counts each sample as the share of a decode step it covers."""
     if dist.rank != 0:
         return None
     w = oda_synth.WORKLOADS[args.workload]
@@ -974,21 +1206,22 @@ def run_reference(args, dist: Dist):
     s = OracleSampler(w, rho, dev, chunks=16)
     for i in range(max(args.warmup, 3)):
         s.sample(i)
-    wall = time.perf_counter()
-    total = sum(s.sample(i) for i in range(args.steps))
-    wall = time.perf_counter() - wall
-    value = w.batch * args.steps / total
+    t0 = time.perf_counter()
+    samples = [s.sample(i) for i in range(args.steps)]
+    wall = time.perf_counter() - t0
+    tokens = sum(w.batch * sw / whole for sw, whole in samples)   # share of a step each covers
+    value = tokens / wall
     cores = _blas_threads()
     sample = ("each step: one oracle sample of a %s decode step (Local at one layer, recall, "
-              "Full at one layer for one KV head over 1/16 of the history) extrapolated to %d "
-              "layers, %d KV heads, the whole history and rho=%.3f"
-              % (w.name, w.layers, w.num_kv_heads, rho))
+              "Full at one layer for one KV head over 1/16 of the history), counted as the "
+              "share of a whole step (%d layers, %d KV heads, the whole history, rho=%.3f) that "
+              "its work covers; %.1f s wall" % (w.name, w.layers, w.num_kv_heads, rho, wall))
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world,
-            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total / args.steps,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * wall / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": w.name, "rho": rho},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": sample + "; %.1f s wall" % wall},
+                             "host_cores": os.cpu_count(), "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -1052,13 +1285,14 @@ def main():
             res = run_reference(args, dist)
         else:
             res, setup = run_oda(args, dist)
-            if (dist.rank == 0 and dist.world == 1 and setup is not None
+            if (dist.rank == 0 and dist.world == 1 and "config" in res
                     and not (args.no_cpu_baseline or args.quick)):
-                rho = res["config"]["rho_realised"]
+                rho = res["config"].get("rho_realised") or 0.5
                 del setup
                 torch.cuda.empty_cache()
                 res["cpu_baseline"] = cpu_baseline(oda_synth.WORKLOADS[args.workload], rho,
                                                    "cuda:%d" % dist.local)
+                res["cpu_baseline_full_run"] = cpu_baseline_full()
         if res is not None and dist.rank == 0:
             print(json.dumps(res), flush=True)
     finally:

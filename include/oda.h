@@ -146,11 +146,13 @@ int oda_decode_full(const oda_kv* kv, const void* q, int32_t num_q_heads, float 
  * allocation failure mid-step, cannot hand in a cudaMalloc'd buffer. The split partials and
  * merge tickets then live in a 2 MiB device array inside liboda, held by every GPU that loads
  * the library until exit; a batch whose workspace (oda_decode_workspace_size) exceeds 2 MiB
- * returns ODA_ERR_WORKSPACE_TOO_SMALL. The first call on each device looks up the array's
- * device address (cudaGetSymbolAddress), so make that first call before any stream capture.
- * Each call clears the array's tickets with an asynchronous memset on `stream` and allocates
- * nothing. All calls share the one array: calls that overlap on the GPU (different streams,
- * no ordering between them) race and give wrong results. */
+ * returns ODA_ERR_WORKSPACE_TOO_SMALL. Every call looks up the array's device address in the
+ * current context (cudaGetSymbolAddress); the first call on a device may load the module, so
+ * make that first call before any stream capture. Every host-side check runs before anything
+ * is queued: a rejected call queues no work. An accepted call clears the array's tickets with
+ * an asynchronous memset on `stream`, then launches; it allocates nothing. All calls share the
+ * one array: calls that overlap on the GPU (different streams, no ordering between them) race
+ * and give wrong results. */
 int oda_decode_full_noalloc(const oda_kv* kv, const void* q, int32_t num_q_heads, float scale,
                             const int32_t* gate, const void* k_new, const void* v_new,
                             void* out, int32_t out_dtype, float* lse, void* stream);
@@ -281,8 +283,10 @@ int oda_recall_loss_grad(const float* h_prev, const float* emb, const void* h_lo
  *      the FP32 recall head and the conditional Full recompute in one GPU execution stream,
  *      e.g. CUDA Graphs) ----------------------------------------------------------------
  * The graph runs, per launch: Local (with commit) at every layer; the recall head on the last
- * layer's Local output; then, inside a conditional IF node that the recall head opens only
- * when some sequence is gated, Full (with gated commit) at every layer.
+ * layer's Local output; then Full (with gated commit) at every layer, either inside a
+ * conditional IF node that the recall head opens only when some sequence is gated
+ * (use_conditional = 1) or as kernels that skip ungated sequences on the device -- with the
+ * persistent step kernels, one launch that returns at once when none is gated.
  * All pointers are captured at creation: the caller refreshes the buffers' contents (seq_lens
  * advanced by one, new q/k/v, new embedding) between launches. */
 typedef struct oda_step_graph oda_step_graph;
@@ -335,10 +339,20 @@ typedef struct {
                                           (the recall head does not run; q_out untouched)    */
   const float* gate_u;                 /* RANDOM: device fp32 [batch], refreshed per step    */
   float rho;                           /* RANDOM: Full-call rate in [0, 1]                   */
+  int32_t step_kernels;                /* ODA_STEP_PERSISTENT: where the step's shape allows,
+                                          Local at every layer plus the gate is ONE launch
+                                          (one 16-CTA cluster per (sequence, KV head), at most
+                                          one CTA per SM; every layer restricted to sink +
+                                          window of at most 144 pages; <= 40 layers; fused
+                                          recall head for batch <= 8, mlp <= 288), and Full at
+                                          every layer is ONE launch that returns at once when
+                                          no sequence is gated; other shapes fall back to
+                                          ODA_STEP_PER_LAYER: one launch per layer and phase */
 } oda_step_desc;
 
 enum { ODA_PHASE_LOCAL = 1, ODA_PHASE_RECALL = 2, ODA_PHASE_FULL = 4 };
 enum { ODA_GATE_RECALL = 0, ODA_GATE_RANDOM = 1 };
+enum { ODA_STEP_PERSISTENT = 0, ODA_STEP_PER_LAYER = 1 };
 
 int oda_step_graph_create(const oda_step_desc* desc, void* stream, oda_step_graph** graph);
 int oda_step_graph_launch(oda_step_graph* graph, void* stream);
@@ -346,7 +360,41 @@ int oda_step_graph_launch(oda_step_graph* graph, void* stream);
  * done, Full done) at caller-created cudaEvent_t handles for the next launches. */
 int oda_step_graph_set_events(oda_step_graph* graph, void* ev_start, void* ev_local,
                               void* ev_recall, void* ev_end);
+/* Limits of the persistent Local kernel on the current device: how many of its 16-CTA
+ * clusters (one per sequence and KV head of a step) the device holds at once for query
+ * heads per KV head `group` (1, 2 or 4), `batch` sequences and a fused recall head of width
+ * `mlp` (0: none), and whether its launches are cooperative (1) or rely on that residency (0).
+ * A step whose batch x KV heads exceeds max_clusters runs Local one launch per layer. */
+int oda_step_kernel_limits(int32_t group, int32_t batch, int32_t mlp, int32_t* max_clusters,
+                           int32_t* cooperative);
+
+/* Kernel launches per step of the graph, by phase: Local (the fused gate included), the gate
+ * kernel (0 when fused), Full (counted as in a step whose Full phase runs). */
+int oda_step_graph_kernels(const oda_step_graph* graph, int32_t* local_launches,
+                           int32_t* gate_launches, int32_t* full_launches);
 void oda_step_graph_destroy(oda_step_graph* graph);
+
+/* ---- test hooks (no counterpart in the papers): exercise the bounded device waits -------
+ * Every device wait of liboda (a copy into shared memory, a count published by other CTAs of
+ * the same launch) gives up after a limit, reports ODA_DEV_TIMEOUT in dev_status and lets the
+ * kernel return. These process-wide settings apply to launches (and step graphs) made after
+ * the call; they exist so that tests can make a wait run out without faulting anything.
+ * oda_debug_set_wait_limit: the limit in ns (0 restores the default of 1 s).
+ * oda_debug_set_stall: ODA_STALL_DECODE_RING makes one stage of CTA 0's first warp in each
+ * split decode launch wait for bytes that no copy delivers; ODA_STALL_LOCAL_CHAIN makes the
+ * first cluster of the persistent Local kernel withhold its layer-0 count; ODA_STALL_FULL_CHAIN
+ * makes CTA 0 of the persistent Full kernel withhold its layer-0 arrival. ODA_STALL_NONE (the
+ * default) turns the hook off. After a timeout the decode workspace must be zero-filled again.
+ * Both return ODA_OK, or ODA_ERR_INVALID_ARG for an unknown kind. */
+enum { ODA_STALL_NONE = 0, ODA_STALL_DECODE_RING = 1, ODA_STALL_LOCAL_CHAIN = 2,
+       ODA_STALL_FULL_CHAIN = 3 };
+int oda_debug_set_wait_limit(unsigned long long ns);
+int oda_debug_set_stall(int kind);
+/* Tuning hook: the shape of the persistent Local kernel in step graphs created after the call:
+ * 0 = 16-CTA clusters of 9 warps (two CTAs per SM), 1 = 14 x 10, 2 = 12 x 11 (one CTA per SM);
+ * -1 (the default) = the first of 1, 2, 0 that covers the step's pages and fits the device.
+ * ODA_OK, or ODA_ERR_INVALID_ARG for another value. */
+int oda_debug_set_local_shape(int index);
 
 #ifdef __cplusplus
 }

@@ -21,9 +21,9 @@ OBJDIR = os.path.join(ROOT, "_build")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "liboda.so")
 
-SOURCES = ["oda_decode.cu", "oda_append.cu", "oda_recall.cu", "oda_graph.cu", "oda_noalloc.cu",
+SOURCES = ["oda_decode.cu", "oda_chain.cu", "oda_append.cu", "oda_recall.cu", "oda_graph.cu", "oda_noalloc.cu",
            "oda_merge.cu", "oda_schedule.cu", "oda_train.cu", "oda_api.cpp"]
-HEADERS = ["oda_common.cuh", "oda_plan.cuh", "oda_internal.h", "oda_recall.cuh"]
+HEADERS = ["oda_common.cuh", "oda_plan.cuh", "oda_internal.h", "oda_recall.cuh", "oda_decode.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-I" + INCLUDE, "-I" + CSRC]
 

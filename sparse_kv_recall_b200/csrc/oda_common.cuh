@@ -81,15 +81,16 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
-// Wait for a barrier phase, giving up after kWaitNs. Returns false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Wait for a barrier phase, giving up after limit_ns. Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -139,12 +140,111 @@ __device__ __forceinline__ void dsmem_st(float* local, unsigned rank, float v) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
+// 16-byte store to the shared memory of CTA `rank` (`local` 16-byte aligned).
+__device__ __forceinline__ void dsmem_st4(float* local, unsigned rank, float4 v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(remote), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+// The shared::cluster address of a variable of this CTA's shared memory in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* local, unsigned rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  return remote;
+}
+// Bulk copy from this CTA's shared memory to a CTA of the cluster (addresses from
+// cluster_addr), completing `bytes` on that CTA's mbarrier (16-byte aligned, multiple of 16).
+__device__ __forceinline__ void bulk_to_cluster(uint32_t dst, const void* src, uint32_t bytes,
+                                                uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "r"(smem_addr(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// Arrive (release, cluster scope) on an mbarrier of a CTA of the cluster (address from
+// cluster_addr). A copy into another CTA's shared memory completes only on that CTA's
+// mbarrier -- bulk async-groups do not track it -- so the receiver tells the sender this way
+// that the sender's source buffer may be written again.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar)
+               : "memory");
+}
+// Wait (bounded) for a phase of this CTA's mbarrier that copies from other CTAs of the cluster
+// complete: acquire at cluster scope. Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  unsigned long long limit_ns) {
+  auto try_wait = [&]() {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+  };
+  if (try_wait()) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (try_wait()) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
 __device__ __forceinline__ float dsmem_ld(const float* local, unsigned rank) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote));
   return v;
+}
+
+// ---- global counters between the CTAs of one launch (persistent kernels) ---------------
+// Release-add by one thread after a CTA barrier publishes the CTA's earlier global writes;
+// an acquire load that sees the count makes them visible to the loading thread, and a CTA
+// barrier after it to the rest of its CTA.
+__device__ __forceinline__ void counter_release_add(unsigned* c, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(c), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned counter_acquire_load(const unsigned* c) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+  return v;
+}
+
+// Spin (one thread) until *c >= target (counts compared modulo 2^32), *abort becomes non-zero
+// or limit_ns pass. Returns 1 when the count was reached, 0 on abort or timeout; the caller
+// raises the abort word on a timeout so that every other waiter of the launch stops at once.
+__device__ __forceinline__ unsigned counter_relaxed_load(const unsigned* c) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acquire_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+// (polls with relaxed loads; the fence after the count is seen gives the acquire)
+__device__ __forceinline__ int counter_wait(const unsigned* c, unsigned target,
+                                            const unsigned* abort, unsigned long long limit_ns) {
+  if ((int)(counter_relaxed_load(c) - target) >= 0) {
+    fence_acquire_gpu();
+    return 1;
+  }
+  const unsigned long long t0 = global_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if ((int)(counter_relaxed_load(c) - target) >= 0) {
+        fence_acquire_gpu();
+        return 1;
+      }
+    if (counter_relaxed_load(abort) != 0u) return 0;
+    if (global_ns() - t0 > limit_ns) return 0;
+  }
 }
 
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {

@@ -25,6 +25,8 @@ struct oda_step_graph {
   cudaEvent_t placeholder[4] = {nullptr, nullptr, nullptr, nullptr};
   cudaGraphNode_t ev_node[4] = {nullptr, nullptr, nullptr, nullptr};
   bool timing = false;
+  int launches[3] = {0, 0, 0};  // kernels per step: Local, gate, Full
+  oda::LocalChainPlan lplan;    // the persistent Local kernel's plan (decided before capture)
 };
 
 namespace {
@@ -59,13 +61,28 @@ int layer_window(const oda_step_desc* d, int l) { return d->windows ? d->windows
 int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditionalHandle cond) {
   const int L = d->num_layers;
   const int phases = d->phases ? d->phases : (ODA_PHASE_LOCAL | ODA_PHASE_RECALL | ODA_PHASE_FULL);
+  const bool persistent = d->step_kernels != ODA_STEP_PER_LAYER;
+  const unsigned long long cond_u64 = d->use_conditional ? (unsigned long long)cond : 0ull;
   int rc;
   if (g->timing && (rc = record_event_node(g, 0)) != ODA_OK) return rc;
+
+  // Local (and, fused into the same launch, the gate) as one persistent kernel when the step's
+  // shape fits it; otherwise one launch per layer and a separate gate kernel.
+  bool gate_done = false;
+  bool local_done = !(phases & ODA_PHASE_LOCAL);
+  if (!local_done && persistent && g->lplan.usable) {
+    // with the gate fused if its shape allows, else Local alone and the gate kernel after it
+    rc = oda::launch_local_chain(d, g->lplan, phases, cond_u64, g->cap);
+    if (rc != ODA_OK) return rc;
+    local_done = true;
+    gate_done = g->lplan.gate_fused && (phases & ODA_PHASE_RECALL) != 0;
+    g->launches[0] = 1;
+  }
   // Programmatic dependent launch between consecutive kernels: each Local layer after the
   // first, the recall head after the last Local layer and each Full layer after the first
   // may start while its predecessor finishes (see the kernels for what they do before
   // waiting). Kernels next to a timing-event node keep ordinary launches.
-  for (int l = 0; l < L && (phases & ODA_PHASE_LOCAL); ++l) {
+  for (int l = 0; l < L && !local_done; ++l) {
     const bool restricted = d->local_layers == nullptr || d->local_layers[l] != 0;
     oda_visibility vis = oda::visibility(restricted ? ODA_MODE_LOCAL : ODA_MODE_FULL);
     vis.sink = layer_sink(d, l);
@@ -75,6 +92,7 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
                             d->lse ? d->lse[l] : nullptr, d->decode_ws, d->decode_ws_bytes,
                             g->cap, l > 0 ? 1 : 0, 0);
     if (rc != ODA_OK) return rc;
+    ++g->launches[0];
   }
   if (g->timing && (rc = record_event_node(g, 1)) != ODA_OK) return rc;
   if (!(phases & ODA_PHASE_RECALL)) {
@@ -83,18 +101,20 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
         if ((rc = record_event_node(g, i)) != ODA_OK) return rc;
     return ODA_OK;
   }
-  const unsigned long long cond_u64 = d->use_conditional ? (unsigned long long)cond : 0ull;
-  if (d->gate_source == ODA_GATE_RANDOM) {
-    rc = oda::launch_gate_schedule(d->gate_u, d->layers[0].batch, d->rho, d->gate_out,
-                                   d->full_count, cond_u64, g->cap);
-  } else {
-    const int hidden = d->num_q_heads * d->layers[0].head_dim;
-    rc = oda::launch_recall(d->h_prev, d->emb, d->out[L - 1], ODA_F32, d->layers[0].batch,
-                            hidden, d->mlp, d->w1, d->b1, d->w2, d->b2, d->theta, d->q_out,
-                            d->gate_out, d->full_count, cond_u64, d->recall_ws,
-                            d->recall_ws_bytes, g->cap, g->timing ? 0 : 1);
+  if (!gate_done) {
+    if (d->gate_source == ODA_GATE_RANDOM) {
+      rc = oda::launch_gate_schedule(d->gate_u, d->layers[0].batch, d->rho, d->gate_out,
+                                     d->full_count, cond_u64, g->cap);
+    } else {
+      const int hidden = d->num_q_heads * d->layers[0].head_dim;
+      rc = oda::launch_recall(d->h_prev, d->emb, d->out[L - 1], ODA_F32, d->layers[0].batch,
+                              hidden, d->mlp, d->w1, d->b1, d->w2, d->b2, d->theta, d->q_out,
+                              d->gate_out, d->full_count, cond_u64, d->recall_ws,
+                              d->recall_ws_bytes, g->cap, g->timing ? 0 : 1);
+    }
+    if (rc != ODA_OK) return rc;
+    g->launches[1] = 1;
   }
-  if (rc != ODA_OK) return rc;
   if (g->timing && (rc = record_event_node(g, 2)) != ODA_OK) return rc;
 
   if (!(phases & ODA_PHASE_FULL)) {
@@ -126,21 +146,29 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
       return ODA_ERR_CUDA;
     full_stream = g->cap_body;
   }
-  for (int l = 0; l < L; ++l) {
-    // The first Full kernel reads the gate the recall head just wrote: inside the IF body it
-    // is the body's first node; without the IF node it waits for the recall head at once.
-    int pdl = 1, wait_first = 0;
-    if (l == 0) {
-      pdl = (!d->use_conditional && !g->timing) ? 1 : 0;
-      wait_first = 1;
+  // Full at every layer: one persistent launch that returns at once when no sequence is gated
+  // (the device-side early exit), or one launch per layer that skips ungated sequences.
+  rc = persistent ? oda::launch_full_chain(d, full_stream) : ODA_ERR_NOT_IMPLEMENTED;
+  if (rc == ODA_OK) g->launches[2] = 1;
+  if (rc == ODA_ERR_NOT_IMPLEMENTED) {
+    rc = ODA_OK;
+    for (int l = 0; l < L; ++l) {
+      // The first Full kernel reads the gate the gate kernel just wrote: inside the IF body it
+      // is the body's first node; without the IF node it waits for the gate kernel at once.
+      int pdl = 1, wait_first = 0;
+      if (l == 0) {
+        pdl = (!d->use_conditional && !g->timing && !gate_done) ? 1 : 0;
+        wait_first = 1;
+      }
+      oda_visibility vis = oda::visibility(ODA_MODE_FULL);
+      vis.gate = d->gate_out;
+      rc = oda::launch_decode(&d->layers[l], vis, d->q_full[l], d->num_q_heads, d->scale,
+                              d->k_full[l], d->v_full[l], d->out[l], ODA_F32,
+                              d->lse ? d->lse[l] : nullptr,
+                              d->decode_ws, d->decode_ws_bytes, full_stream, pdl, wait_first);
+      if (rc != ODA_OK) break;
+      ++g->launches[2];
     }
-    oda_visibility vis = oda::visibility(ODA_MODE_FULL);
-    vis.gate = d->gate_out;
-    rc = oda::launch_decode(&d->layers[l], vis, d->q_full[l], d->num_q_heads, d->scale,
-                            d->k_full[l], d->v_full[l], d->out[l], ODA_F32,
-                            d->lse ? d->lse[l] : nullptr,
-                            d->decode_ws, d->decode_ws_bytes, full_stream, pdl, wait_first);
-    if (rc != ODA_OK) break;
   }
   if (d->use_conditional) {
     cudaGraph_t done = nullptr;
@@ -173,6 +201,8 @@ int check_desc(const oda_step_desc* d) {
   if (d->gate_source == ODA_GATE_RANDOM &&
       (d->gate_u == nullptr || !(d->rho >= 0.f && d->rho <= 1.f)))
     return ODA_ERR_INVALID_ARG;
+  if (d->step_kernels != ODA_STEP_PERSISTENT && d->step_kernels != ODA_STEP_PER_LAYER)
+    return ODA_ERR_INVALID_ARG;
   return ODA_OK;
 }
 
@@ -186,6 +216,7 @@ extern "C" int oda_step_graph_create(const oda_step_desc* desc, void* stream,
   int rc = check_desc(desc);
   if (rc != ODA_OK) return rc;
   if ((rc = oda::prepare_decode_kernels()) != ODA_OK) return rc;
+  if ((rc = oda::prepare_chain_kernels()) != ODA_OK) return rc;
   oda_step_graph* g = new (std::nothrow) oda_step_graph();
   if (g == nullptr) return ODA_ERR_CUDA;
   g->timing = desc->timing_events != 0;
@@ -208,6 +239,11 @@ extern "C" int oda_step_graph_create(const oda_step_desc* desc, void* stream,
           cudaSuccess) {
     release(g);
     return ODA_ERR_CUDA;
+  }
+  const int all = ODA_PHASE_LOCAL | ODA_PHASE_RECALL | ODA_PHASE_FULL;
+  if ((rc = oda::plan_local_chain(desc, desc->phases ? desc->phases : all, &g->lplan)) != ODA_OK) {
+    release(g);
+    return rc;
   }
   if (cudaStreamBeginCaptureToGraph(g->cap, g->graph, nullptr, nullptr, 0,
                                     cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
@@ -243,6 +279,17 @@ extern "C" int oda_step_graph_set_events(oda_step_graph* graph, void* ev_start, 
                                              static_cast<cudaEvent_t>(evs[i])) != cudaSuccess)
       return ODA_ERR_CUDA;
   }
+  return ODA_OK;
+}
+
+extern "C" int oda_step_graph_kernels(const oda_step_graph* graph, int32_t* local_launches,
+                                      int32_t* gate_launches, int32_t* full_launches) {
+  if (graph == nullptr || local_launches == nullptr || gate_launches == nullptr ||
+      full_launches == nullptr)
+    return ODA_ERR_INVALID_ARG;
+  *local_launches = graph->launches[0];
+  *gate_launches = graph->launches[1];
+  *full_launches = graph->launches[2];
   return ODA_OK;
 }
 

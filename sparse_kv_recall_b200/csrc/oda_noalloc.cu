@@ -7,8 +7,7 @@
 // cudaMalloc can imply in the middle of a decode step. For them, the split partials and
 // merge tickets of the Full decode live in one file-scope device array. Every GPU that
 // loads this library holds that array (2 MiB) until the process exits.
-#include "oda_common.cuh"
-#include "oda_internal.h"
+#include "oda_decode.cuh"
 
 namespace oda {
 namespace {
@@ -16,20 +15,17 @@ namespace {
 constexpr size_t kStaticWsBytes = size_t(2) << 20;  // 2 MiB of scratch per device
 __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
 
-// Device address of g_static_ws on the current device, looked up once per device with that
-// device current. In host code the symbol itself is only a host-side stand-in: passing it
-// to a kernel would fault, or silently touch the wrong memory where the GPU can reach host
-// memory, so only this looked-up address is ever handed to the kernel.
+// Device address of g_static_ws in the current device's context. In host code the symbol
+// itself is only a host-side stand-in: passing it to a kernel would fault, or silently touch
+// the wrong memory where the GPU can reach host memory, so only this looked-up address is
+// ever handed to the kernel. It is looked up on every call (a cheap host call once the module
+// is loaded) rather than cached: a cache would go stale if the context were torn down and
+// created again (the module, and the array, could then sit elsewhere), and a cache shared by
+// host threads would need its own synchronisation.
 int static_ws_address(void** ptr) {
-  static void* addr[64] = {nullptr};
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ODA_ERR_CUDA;
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) return ODA_ERR_CUDA;
-    addr[dev] = p;
-  }
-  *ptr = addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) return ODA_ERR_CUDA;
+  *ptr = p;
   return ODA_OK;
 }
 
@@ -50,12 +46,18 @@ extern "C" int oda_decode_full_noalloc(const oda_kv* kv, const void* q, int32_t 
   if (total > oda::kStaticWsBytes) return ODA_ERR_WORKSPACE_TOO_SMALL;
   void* ws = nullptr;
   if ((rc = oda::static_ws_address(&ws)) != ODA_OK) return rc;
+  oda_visibility vis = oda::visibility(ODA_MODE_FULL);
+  vis.gate = gate;
+  // Every host-side check of the launch first, so that a rejected call queues no work at all
+  // (no stray write to the shared array, no stray node in a graph being captured).
+  oda::DecodeParams p;
+  if ((rc = oda::decode_params(kv, vis, q, num_q_heads, scale, k_new, v_new, out, out_dtype, lse,
+                               ws, oda::kStaticWsBytes, &p)) != ODA_OK)
+    return rc;
   // The array keeps whatever the previous call left; the merge tickets must start at zero.
   if (cudaMemsetAsync(static_cast<unsigned char*>(ws) + ticket_off, 0, total - ticket_off,
                       static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ODA_ERR_CUDA;
-  oda_visibility vis = oda::visibility(ODA_MODE_FULL);
-  vis.gate = gate;
   return oda::launch_decode(kv, vis, q, num_q_heads, scale, k_new, v_new, out, out_dtype, lse,
                             ws, oda::kStaticWsBytes, stream, 0, 0);
 }

@@ -249,6 +249,16 @@ int launch_recall(const float* h_prev, const float* emb, const void* h_local, in
 
 using namespace oda;
 
+namespace oda {
+int recall_ws_tickets(int batch, int hidden, int mlp, size_t* ticket_off, int* tiles) {
+  if (batch < 0 || hidden < 1 || mlp < kColTile || mlp % kColTile != 0) return ODA_ERR_INVALID_ARG;
+  const RecallWs w = recall_ws(batch, hidden, mlp);
+  *ticket_off = w.ticket_off;
+  *tiles = w.tiles;
+  return ODA_OK;
+}
+}  // namespace oda
+
 extern "C" int oda_recall_workspace_size(int32_t batch, int32_t hidden, int32_t mlp,
                                          size_t* bytes) {
   if (bytes == nullptr || batch < 0 || hidden < 1 || mlp < kColTile || mlp % kColTile != 0)

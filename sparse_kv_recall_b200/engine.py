@@ -78,7 +78,8 @@ class OdaEngine:
                  timing: bool = False, local_layers: Optional[Sequence[int]] = None,
                  sinks: Optional[Sequence[int]] = None, windows: Optional[Sequence[int]] = None,
                  random_rho: Optional[float] = None,
-                 with_lse: bool = False, with_stats: bool = True, phases: int = 0):
+                 with_lse: bool = False, with_stats: bool = True, phases: int = 0,
+                 step_kernels: int = oda.ODA_STEP_PERSISTENT):
         self.L = len(k_caches)
         self.B = block_table.shape[0]
         self.hq = num_q_heads
@@ -92,6 +93,7 @@ class OdaEngine:
         self.phases = phases
         self.local_layers, self.sinks, self.windows = local_layers, sinks, windows
         self.random_rho = random_rho   # not None: random gate schedule at this rate
+        self.step_kernels = step_kernels
         dev = block_table.device
         self.layout = StagingLayout(self.L, self.B, self.hq, self.hkv, self.hidden)
         self.staging = torch.zeros(self.layout.nbytes, dtype=torch.uint8, device=dev)
@@ -147,7 +149,7 @@ class OdaEngine:
                 gate_u=v["gate_u"] if self.random_rho is not None else None,
                 rho=self.random_rho or 0.0,
                 use_conditional=self.use_conditional, timing_events=self.timing,
-                phases=phases))
+                phases=phases, step_kernels=self.step_kernels))
         return graphs
 
     def set_h_prev(self, h0: torch.Tensor, step: int = 0):

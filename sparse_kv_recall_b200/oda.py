@@ -43,6 +43,12 @@ ODA_PHASE_RECALL = 2
 ODA_PHASE_FULL = 4
 ODA_GATE_RECALL = 0
 ODA_GATE_RANDOM = 1
+ODA_STEP_PERSISTENT = 0
+ODA_STEP_PER_LAYER = 1
+ODA_STALL_NONE = 0
+ODA_STALL_DECODE_RING = 1
+ODA_STALL_LOCAL_CHAIN = 2
+ODA_STALL_FULL_CHAIN = 3
 
 
 class OdaError(RuntimeError):
@@ -96,6 +102,7 @@ class oda_step_desc(ctypes.Structure):
         ("use_conditional", ctypes.c_int32), ("timing_events", ctypes.c_int32),
         ("phases", ctypes.c_int32), ("gate_source", ctypes.c_int32),
         ("gate_u", ctypes.c_void_p), ("rho", ctypes.c_float),
+        ("step_kernels", ctypes.c_int32),
     ]
 
 
@@ -134,6 +141,12 @@ _SIGNATURES = {
     "oda_step_graph_launch": (ctypes.c_int, [_P, _P]),
     "oda_step_graph_set_events": (ctypes.c_int, [_P, _P, _P, _P, _P]),
     "oda_step_graph_destroy": (None, [_P]),
+    "oda_step_graph_kernels": (ctypes.c_int, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I),
+                                              ctypes.POINTER(_I)]),
+    "oda_step_kernel_limits": (ctypes.c_int, [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
+    "oda_debug_set_wait_limit": (ctypes.c_int, [ctypes.c_ulonglong]),
+    "oda_debug_set_stall": (ctypes.c_int, [ctypes.c_int]),
+    "oda_debug_set_local_shape": (ctypes.c_int, [ctypes.c_int]),
 }
 
 
@@ -369,7 +382,8 @@ class StepGraph:
                  h_prev, emb, w1, b1, w2, b2: float, theta: float, q_out, gate_out,
                  decode_ws, recall_ws, full_count=None, lse=None, local_layers=None,
                  sinks=None, windows=None, use_conditional: bool = True,
-                 timing_events: bool = False, phases: int = 0, gate_u=None, rho: float = 0.0):
+                 timing_events: bool = False, phases: int = 0, gate_u=None, rho: float = 0.0,
+                 step_kernels: int = ODA_STEP_PERSISTENT):
         L = len(kvs)
         self._keep = []
         layers = (oda_kv * L)(*kvs)
@@ -411,7 +425,8 @@ class StepGraph:
             use_conditional=int(bool(use_conditional)), timing_events=int(bool(timing_events)),
             phases=int(phases),
             gate_source=ODA_GATE_RANDOM if gate_u is not None else ODA_GATE_RECALL,
-            gate_u=_ptr(gate_u, torch.float32, "gate_u"), rho=float(rho))
+            gate_u=_ptr(gate_u, torch.float32, "gate_u"), rho=float(rho),
+            step_kernels=int(step_kernels))
         self._desc = d
         h = ctypes.c_void_p(0)
         _check(load().oda_step_graph_create(ctypes.byref(d), None, ctypes.byref(h)),
@@ -420,6 +435,14 @@ class StepGraph:
 
     def launch(self, stream=None):
         _check(load().oda_step_graph_launch(self._h, _stream(stream)), "oda_step_graph_launch")
+
+    def kernels(self):
+        """(Local, gate, Full) kernel launches per step of this graph; the Full count is that
+        of a step whose Full phase runs (with an IF node it is skipped otherwise)."""
+        a, b, c = _I(0), _I(0), _I(0)
+        _check(load().oda_step_graph_kernels(self._h, ctypes.byref(a), ctypes.byref(b),
+                                             ctypes.byref(c)), "oda_step_graph_kernels")
+        return a.value, b.value, c.value
 
     def set_events(self, ev_start, ev_local, ev_recall, ev_end):
         _check(load().oda_step_graph_set_events(self._h, ev_start.cuda_event, ev_local.cuda_event,
@@ -436,6 +459,29 @@ class StepGraph:
             self.close()
         except Exception:
             pass
+
+
+def oda_step_kernel_limits(group: int, batch: int, mlp: int):
+    """(max clusters of the persistent Local kernel resident at once, cooperative launches)."""
+    n, c = _I(0), _I(0)
+    _check(load().oda_step_kernel_limits(int(group), int(batch), int(mlp), ctypes.byref(n),
+                                         ctypes.byref(c)), "oda_step_kernel_limits")
+    return n.value, c.value
+
+
+def oda_debug_set_wait_limit(ns: int):
+    """Test hook: the limit (ns) of every bounded device wait of later launches; 0 = 1 s."""
+    _check(load().oda_debug_set_wait_limit(int(ns)), "oda_debug_set_wait_limit")
+
+
+def oda_debug_set_local_shape(index: int):
+    """Tuning hook: shape of the persistent Local kernel in later step graphs (-1 = automatic)."""
+    _check(load().oda_debug_set_local_shape(int(index)), "oda_debug_set_local_shape")
+
+
+def oda_debug_set_stall(kind: int):
+    """Test hook: make one bounded wait of later launches run out (ODA_STALL_*)."""
+    _check(load().oda_debug_set_stall(int(kind)), "oda_debug_set_stall")
 
 
 def oda_recall_train_workspace_size(batch: int, hidden: int, mlp: int) -> int:

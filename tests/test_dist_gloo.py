@@ -1,6 +1,7 @@
 """The multi-GPU plumbing of bench.py on CPU ranks (gloo, world size 2): each rank runs its
 own replica with its own seeded sequences, timing is the max over ranks, throughput the sum
 of every rank's tokens, and there is no collective on the data path."""
+import json
 import os
 import socket
 
@@ -69,19 +70,35 @@ def test_clock_sampler_without_nvidia_smi_is_reported():
     assert c.stop()["reasons"] == ["nvidia-smi unavailable"]
 
 
-def test_profiled_bytes_follow_committed_summaries(tmp_path, monkeypatch):
-    """bench.py reads the DRAM bytes of the step's kernels from the committed ncu summaries,
-    and only while the kernel sources they were taken on are unchanged."""
+def test_profiled_bytes_follow_committed_captures(tmp_path, monkeypatch):
+    """bench.py reads the DRAM bytes of the step's kernels from the JSON its --ncu-summary
+    writes from an ncu capture, and only while the kernel sources it was taken on are
+    unchanged; the summary is read back from a raw CSV export the way ncu writes it."""
     import bench
-    full = bench.profiled_traffic(131073)
-    assert full is not None and 1.0 <= full / (131073 * 8 * 512) < 1.05
-    step = bench.profiled_step_bytes(28, 2.0, 131073)
-    local = float(bench._profile_fields(bench.LOCAL_PROFILE)["dram_bytes_per_launch"])
-    recall = float(bench._profile_fields(bench.RECALL_PROFILE,
-                                         bench.RECALL_SOURCES)["dram_bytes_per_launch"])
-    assert step == 28 * local + recall + 2.0 * full
-    stale = tmp_path / "stale.md"
-    stale.write_text(open(bench.LOCAL_PROFILE).read().replace(
-        bench.kernel_source_hash(), "0000000000000000"))
-    monkeypatch.setattr(bench, "LOCAL_PROFILE", str(stale))
-    assert bench.profiled_step_bytes(28, 2.0, 131073) is None
+    csv = tmp_path / "raw.csv"
+    csv.write_text(
+        '"ID","Process ID","Kernel Name","dram__bytes_read.sum","dram__bytes_write.sum",'
+        '"gpu__time_duration.sum"\n'
+        '"","","","Mbyte","Mbyte","usecond"\n'
+        '"0","1","void oda::local_chain_kernel<2>(oda::LocalChainParams)","200.5","1.5","40"\n'
+        '"1","1","void oda::full_chain_kernel<2>(oda::FullChainParams)","1,080","8","200"\n'
+        '"2","1","void oda::full_chain_kernel<2>(oda::FullChainParams)","1,082","8","202"\n')
+    full = tmp_path / "full.json"
+    info = bench.ncu_summary(str(csv), "full_chain_kernel", str(full),
+                             {"tokens_per_layer": 131073, "layers_per_launch": 2})
+    assert info["launches_captured"] == 2
+    assert info["dram_bytes_per_launch"] == 1089e6
+    assert abs(info["gpu_time_s_per_launch_under_ncu"] - 201e-6) < 1e-12
+    local = tmp_path / "local.json"
+    bench.ncu_summary(str(csv), "local_chain_kernel", str(local), {"layers_per_launch": 28})
+    monkeypatch.setattr(bench, "PROFILE", str(full))
+    monkeypatch.setattr(bench, "LOCAL_PROFILE", str(local))
+    per = 1089e6 / (131073 * 2)
+    assert abs(bench.profiled_traffic(131073, 28) - per * 131073 * 28) < 1.0
+    step = bench.profiled_step_bytes(28, 0.5, 131073)
+    assert abs(step - (202e6 + 0.5 * per * 131073 * 28)) < 1.0
+    stale = json.load(open(full))
+    stale["source_sha"] = "0000000000000000"
+    json.dump(stale, open(full, "w"))
+    assert bench.profiled_traffic(131073, 28) is None
+    assert bench.profiled_step_bytes(28, 0.5, 131073) is None

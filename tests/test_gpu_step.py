@@ -31,14 +31,16 @@ def _logical(bits, bt, caps, hkv, d):
 
 
 def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02, timing=False,
-               **layer_ranges):
+               step_kernels=oda.ODA_STEP_PERSISTENT, expect_kernels=None, **layer_ranges):
     lay = oda_synth.make_layout(w, extra_tokens=steps + 2, device="cuda", lengths=lengths)
     caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
     rw = oda_synth.make_recall_weights(w, device="cuda", std=recall_std)
     eng = OdaEngine([c[0] for c in caches], [c[1] for c in caches], lay.block_table,
                     w.num_q_heads, (rw.w1, rw.b1, rw.w2, rw.b2), theta, sink=w.sink,
                     window=w.window, use_conditional=use_conditional, timing=timing,
-                    **layer_ranges)
+                    step_kernels=step_kernels, **layer_ranges)
+    if expect_kernels is not None:                  # launches per step: Local, gate, Full
+        assert eng.graphs[0].kernels() == expect_kernels, eng.graphs[0].kernels()
     h0 = oda_synth.make_h0(w, device="cuda")
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     for e in evs:
@@ -180,3 +182,115 @@ def test_local_only_phase_graph():
         for b, n in enumerate(lengths):
             assert np.array_equal(dk[b, :, :n + 2], dec.k[l][b, :, :n + 2])
     eng.close()
+
+
+# ---- the persistent step kernels: Local at every layer + fused gate as one launch (one
+# cluster per (sequence, KV head), batch x KV heads <= 9 clusters), Full as one launch ----
+
+def _expected_kernels(w):
+    """(Local, gate, Full) launches per step the step graph should take on this device: the
+    persistent Local kernel with the fused gate when its clusters fit, without it when only
+    the smaller shared-memory form fits, else one launch per layer and a gate kernel."""
+    G, ncl = w.num_q_heads // w.num_kv_heads, w.batch * w.num_kv_heads
+    fused, _ = oda.oda_step_kernel_limits(G, w.batch, w.mlp)
+    plain, _ = oda.oda_step_kernel_limits(G, w.batch, 0)
+    if fused >= ncl:
+        return (1, 0, 1)
+    if plain >= ncl:
+        return (1, 1, 1)
+    return (w.layers, 1, 1)
+
+
+def test_persistent_local_kernel_serves_the_default_shape():
+    """Batch 1 x 8 KV heads with two query heads each (the long-context workload's shape) must
+    fit the persistent Local kernel with its fused gate."""
+    clusters, coop = oda.oda_step_kernel_limits(2, 1, 256)
+    assert clusters >= 8, clusters
+
+
+@pytest.mark.parametrize("use_conditional", [False, True])
+@pytest.mark.parametrize("hq,hkv,batch,lengths", [
+    (16, 8, 1, [700]),                 # G = 2, the default workload's grouping
+    (32, 8, 1, [333]),                 # G = 4 (8 clusters of one CTA per SM: may not fit)
+    (8, 8, 1, [512]),                  # G = 1
+    (8, 4, 2, [700, 45]),              # two sequences, one shorter than the window
+    (4, 2, 4, [300, 129, 1000, 16]),   # four sequences
+    (8, 4, 1, [2000]),                 # four KV heads: fewer clusters than the maximum
+])
+def test_persistent_step_kernels_match_oracle(use_conditional, hq, hkv, batch, lengths):
+    w = oda_synth.Workload(name="chain", layers=3, batch=batch, num_q_heads=hq,
+                           num_kv_heads=hkv, prefill=max(lengths), steps=5, seed=90 + hq + batch,
+                           sink=4, window=128)
+    n = _run_steps(w, lengths, 5, theta=0.0, use_conditional=use_conditional,
+                   expect_kernels=_expected_kernels(w))
+    assert 0 < n < 5 * batch
+
+
+def test_persistent_step_kernels_per_layer_sink_and_window():
+    w = oda_synth.Workload(name="chain-ranges", layers=3, batch=1, num_q_heads=16,
+                           num_kv_heads=8, prefill=900, steps=4, seed=93, sink=4, window=64)
+    _run_steps(w, [900], 4, theta=0.0, sinks=[4, 0, 16], windows=[64, 17, 2000],
+               expect_kernels=(1, 0, 1))
+
+
+def test_persistent_step_kernels_random_schedule_and_ends():
+    w = oda_synth.Workload(name="chain-random", layers=2, batch=1, num_q_heads=16,
+                           num_kv_heads=8, prefill=400, steps=6, seed=94, sink=4, window=64)
+    _run_steps(w, [400], 6, theta=0.0, random_rho=0.5, expect_kernels=(1, 0, 1))
+    assert _run_steps(w, [400], 3, theta=float("inf"), expect_kernels=(1, 0, 1)) == 0
+    assert _run_steps(w, [400], 3, theta=-float("inf"), expect_kernels=(1, 0, 1)) == 3
+
+
+def test_persistent_step_kernels_with_timing_events():
+    w = oda_synth.Workload(name="chain-timing", layers=2, batch=1, num_q_heads=16,
+                           num_kv_heads=8, prefill=600, steps=3, seed=95, sink=4, window=256)
+    _run_steps(w, [600], 3, theta=0.0, timing=True, expect_kernels=(1, 0, 1))
+
+
+def test_shapes_outside_the_persistent_local_kernel_fall_back():
+    """Batch 3 x 8 KV heads needs more clusters than the GPU holds at once: Local runs per
+    layer with the recall kernel after it, Full still as one persistent launch."""
+    w = oda_synth.Workload(name="chain-fallback", layers=2, batch=3, num_q_heads=16,
+                           num_kv_heads=8, prefill=300, steps=3, seed=96, sink=4, window=64)
+    _run_steps(w, [300, 37, 170], 3, theta=0.0, expect_kernels=(2, 1, 1))
+
+
+@pytest.mark.parametrize("theta", [float("inf"), -float("inf")])
+def test_persistent_step_equals_per_layer(theta):
+    """The persistent Full kernel runs the per-layer split pass itself, so with every step
+    recomputed by Full (theta = -inf) every layer output is bitwise the per-layer launches'.
+    The persistent Local kernel forms its page scores on the tensor cores and merges one state
+    per warp (the per-layer cluster kernel: CUDA-core scores, two states per warp), so Local
+    outputs (theta = +inf) agree to fp32 rounding. Committed K/V bits and the attended-row and
+    page counters are identical either way; theta at +-inf keeps the gate out of it (the fused
+    recall head sums in another order than the recall kernel)."""
+    w = oda_synth.Workload(name="chain-bitwise", layers=3, batch=1, num_q_heads=16,
+                           num_kv_heads=8, prefill=3000, steps=3, seed=97, sink=4, window=512)
+    res = {}
+    for sk in (oda.ODA_STEP_PERSISTENT, oda.ODA_STEP_PER_LAYER):
+        lay = oda_synth.make_layout(w, extra_tokens=5, device="cuda")
+        caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
+        rw = oda_synth.make_recall_weights(w, device="cuda")
+        eng = OdaEngine([c[0] for c in caches], [c[1] for c in caches], lay.block_table,
+                        w.num_q_heads, (rw.w1, rw.b1, rw.w2, rw.b2), theta, sink=w.sink,
+                        window=w.window, use_conditional=False, step_kernels=sk)
+        eng.set_h_prev(oda_synth.make_h0(w, device="cuda"), 0)
+        outs = []
+        for i in range(w.steps):
+            fill_staging(eng.v, oda_synth.make_step_inputs(w, i, device="cuda"),
+                         [w.prefill + i + 1])
+            eng.launch(i)
+            outs.append(torch.stack([eng.layer_out(i, l).clone() for l in range(w.layers)]))
+        torch.cuda.synchronize()
+        assert int(eng.status.item()) == 0
+        res[sk] = (torch.stack(outs).cpu(), [(c[0].cpu(), c[1].cpu()) for c in caches],
+                   eng.stats.cpu())
+        eng.close()
+    a, b = res[oda.ODA_STEP_PERSISTENT], res[oda.ODA_STEP_PER_LAYER]
+    if theta < 0:
+        assert torch.equal(a[0], b[0])
+    else:
+        assert (a[0] - b[0]).abs().max().item() <= 2e-6 * max(1.0, b[0].abs().max().item())
+    for (ka, va), (kb, vb) in zip(a[1], b[1]):
+        assert torch.equal(ka, kb) and torch.equal(va, vb)
+    assert torch.equal(a[2], b[2])                       # rows / pages counters
