@@ -51,6 +51,9 @@ KERNEL_SOURCES = ["oda_decode.cuh", "oda_decode.cu", "oda_chain.cu", "oda_plan.c
                   "oda_common.cuh", "oda_recall.cuh"]
 
 
+STEP_KERNELS = {"full-persistent": 0, "per-layer": 1, "persistent": 2}  # ODA_STEP_*
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -75,13 +78,24 @@ def parse_args():
                     help="put the Full phase behind a graph IF node set by the gate, instead of "
                          "the default device-side early exit of the persistent Full kernel (ncu "
                          "lists kernel nodes only of graphs without conditional nodes)")
-    ap.add_argument("--step-kernels", choices=["persistent", "per-layer"], default="persistent",
-                    help="persistent: Local at every layer with the fused gate, and Full at "
-                         "every layer, as one launch each; per-layer: one launch per layer "
+    ap.add_argument("--step-kernels", choices=sorted(STEP_KERNELS), default="full-persistent",
+                    help="full-persistent: Local one launch per layer, the gate kernel, Full "
+                         "at every layer as one launch; persistent: Local at every layer with "
+                         "the fused gate as one launch too; per-layer: one launch per layer "
                          "and phase")
-    ap.add_argument("--profile-kernel", choices=["full", "local", "recall", "train"],
-                    help="one layer of the workload, the named kernel launched --steps times "
-                         "(a small case for ncu captures); prints nothing")
+    ap.add_argument("--profile-kernel",
+                    choices=["full", "local", "recall", "train", "step"],
+                    help="a small case for ncu captures, launched --steps times; prints "
+                         "nothing. full / local / recall / train: one layer of the workload "
+                         "and the named per-layer kernel; step: the step graph over "
+                         "--profile-layers layers with every step gated (theta = -inf), so "
+                         "that both persistent kernels run")
+    ap.add_argument("--profile-layers", type=int, default=4)
+    ap.add_argument("--ncu-summary", nargs=4, metavar=("CSV", "KERNEL", "OUT", "EXTRA"),
+                    help="write OUT (JSON): the per-launch DRAM bytes of KERNEL's launches in "
+                         "CSV (an `ncu --page raw --csv` export), with the JSON object EXTRA "
+                         "describing one launch (tokens_per_layer, layers_per_launch, ...); "
+                         "needs no GPU")
     return ap.parse_args()
 
 
@@ -838,8 +852,7 @@ def run_oda(args, dist: Dist):
              + (2 * VAR + 16 if VAR else 0))
     s = Setup(w, dist.rank, total, float("inf") if w.theta is None else w.theta, dev,
               use_conditional=args.conditional,
-              step_kernels=oda.ODA_STEP_PER_LAYER if args.step_kernels == "per-layer"
-              else oda.ODA_STEP_PERSISTENT)
+              step_kernels=STEP_KERNELS[args.step_kernels])
     eng = s.eng
     stream = torch.cuda.current_stream()
     step = 0
@@ -1232,8 +1245,11 @@ def run_profile_case(args):
     from sparse_kv_recall_b200 import oda
     B.build()
     oda.load()
-    w = oda_synth.scaled(oda_synth.WORKLOADS[args.workload], layers=1)
     dev = "cuda"
+    if args.profile_kernel == "step":
+        run_profile_step(args, dev)
+        return
+    w = oda_synth.scaled(oda_synth.WORKLOADS[args.workload], layers=1)
     lengths = oda_synth.prefill_lengths(w)
     lay = oda_synth.make_layout(w, extra_tokens=8, device=dev)
     kc, vc = oda_synth.make_kv_cache(w, lay, 0, device=dev)
@@ -1274,8 +1290,34 @@ def run_profile_case(args):
     torch.cuda.synchronize()
 
 
+def run_profile_step(args, dev: str):
+    """The step graph of the workload over --profile-layers layers (KV pages far larger than
+    L2, a few GB), every step gated, launched --steps times on fresh staged inputs."""
+    from sparse_kv_recall_b200.engine import OdaEngine, fill_staging
+    w = oda_synth.scaled(oda_synth.WORKLOADS[args.workload], layers=args.profile_layers)
+    lengths = oda_synth.prefill_lengths(w)
+    lay = oda_synth.make_layout(w, extra_tokens=args.steps + 8, device=dev)
+    caches = [oda_synth.make_kv_cache(w, lay, l, device=dev) for l in range(w.layers)]
+    rw = oda_synth.make_recall_weights(w, device=dev)
+    eng = OdaEngine([c[0] for c in caches], [c[1] for c in caches], lay.block_table,
+                    w.num_q_heads, (rw.w1, rw.b1, rw.w2, rw.b2), -float("inf"), sink=w.sink,
+                    window=w.window, use_conditional=False)
+    eng.set_h_prev(oda_synth.make_h0(w, device=dev), 0)
+    for i in range(args.steps):
+        si = oda_synth.make_step_inputs(w, i, device=dev)
+        fill_staging(eng.v, si, [n + i + 1 for n in lengths])
+        eng.launch(i)
+    torch.cuda.synchronize()
+    assert int(eng.status.item()) == 0, "device status %d" % int(eng.status.item())
+    eng.close()
+
+
 def main():
     args = parse_args()
+    if args.ncu_summary:
+        csv_path, kernel, out, extra = args.ncu_summary
+        print(json.dumps(ncu_summary(csv_path, kernel, out, json.loads(extra))))
+        return
     if args.profile_kernel:
         run_profile_case(args)
         return

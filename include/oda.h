@@ -339,20 +339,24 @@ typedef struct {
                                           (the recall head does not run; q_out untouched)    */
   const float* gate_u;                 /* RANDOM: device fp32 [batch], refreshed per step    */
   float rho;                           /* RANDOM: Full-call rate in [0, 1]                   */
-  int32_t step_kernels;                /* ODA_STEP_PERSISTENT: where the step's shape allows,
-                                          Local at every layer plus the gate is ONE launch
-                                          (one 16-CTA cluster per (sequence, KV head), at most
-                                          one CTA per SM; every layer restricted to sink +
-                                          window of at most 144 pages; <= 40 layers; fused
-                                          recall head for batch <= 8, mlp <= 288), and Full at
-                                          every layer is ONE launch that returns at once when
-                                          no sequence is gated; other shapes fall back to
-                                          ODA_STEP_PER_LAYER: one launch per layer and phase */
+  int32_t step_kernels;                /* ODA_STEP_FULL_PERSISTENT (0, the default): Local one
+                                          launch per layer, the gate kernel, then Full at every
+                                          layer as ONE launch (<= 40 layers) that returns at
+                                          once when no sequence is gated (no IF node needed);
+                                          ODA_STEP_PERSISTENT: as well, where the step's shape
+                                          allows, Local at every layer plus the gate as ONE
+                                          launch (one cluster per (sequence, KV head); every
+                                          layer restricted to sink + window of at most 144
+                                          pages; fused recall head for batch <= 8, mlp a
+                                          multiple of 64 up to 288);
+                                          ODA_STEP_PER_LAYER: one launch per layer and phase.
+                                          A shape outside a persistent kernel's limits runs
+                                          that phase per layer. */
 } oda_step_desc;
 
 enum { ODA_PHASE_LOCAL = 1, ODA_PHASE_RECALL = 2, ODA_PHASE_FULL = 4 };
 enum { ODA_GATE_RECALL = 0, ODA_GATE_RANDOM = 1 };
-enum { ODA_STEP_PERSISTENT = 0, ODA_STEP_PER_LAYER = 1 };
+enum { ODA_STEP_FULL_PERSISTENT = 0, ODA_STEP_PER_LAYER = 1, ODA_STEP_PERSISTENT = 2 };
 
 int oda_step_graph_create(const oda_step_desc* desc, void* stream, oda_step_graph** graph);
 int oda_step_graph_launch(oda_step_graph* graph, void* stream);
@@ -360,11 +364,14 @@ int oda_step_graph_launch(oda_step_graph* graph, void* stream);
  * done, Full done) at caller-created cudaEvent_t handles for the next launches. */
 int oda_step_graph_set_events(oda_step_graph* graph, void* ev_start, void* ev_local,
                               void* ev_recall, void* ev_end);
-/* Limits of the persistent Local kernel on the current device: how many of its 16-CTA
- * clusters (one per sequence and KV head of a step) the device holds at once for query
- * heads per KV head `group` (1, 2 or 4), `batch` sequences and a fused recall head of width
- * `mlp` (0: none), and whether its launches are cooperative (1) or rely on that residency (0).
- * A step whose batch x KV heads exceeds max_clusters runs Local one launch per layer. */
+/* Limits of the persistent Local kernel on the current device: how many of its clusters
+ * (one per sequence and KV head of a step; the most that any of its cluster shapes holds) the
+ * device holds at once for query heads per KV head `group` (1, 2 or 4), `batch` sequences and
+ * a fused recall head of width `mlp` (0: none), and whether its launches are cooperative (1)
+ * or rely on that residency (0). A step whose batch x KV heads exceeds max_clusters runs Local
+ * one launch per layer. The fused recall head also needs batch x KV heads <= the head's row
+ * slabs, ceil(3 hidden / 256) (its per-cluster sums live in the recall workspace); otherwise
+ * the gate runs as its own kernel after the Local launch. */
 int oda_step_kernel_limits(int32_t group, int32_t batch, int32_t mlp, int32_t* max_clusters,
                            int32_t* cooperative);
 
@@ -391,8 +398,9 @@ enum { ODA_STALL_NONE = 0, ODA_STALL_DECODE_RING = 1, ODA_STALL_LOCAL_CHAIN = 2,
 int oda_debug_set_wait_limit(unsigned long long ns);
 int oda_debug_set_stall(int kind);
 /* Tuning hook: the shape of the persistent Local kernel in step graphs created after the call:
- * 0 = 16-CTA clusters of 9 warps (two CTAs per SM), 1 = 14 x 10, 2 = 12 x 11 (one CTA per SM);
- * -1 (the default) = the first of 1, 2, 0 that covers the step's pages and fits the device.
+ * 0 = 16-CTA clusters of 9 warps (two CTAs per SM), 1 = 14 x 10, 2 = 12 x 11, 3 = 8 x 18 (one
+ * CTA per SM; one or two query heads per KV head only); -1 (the default) = the first of 3, 1,
+ * 2, 0 that the group size has, covers the step's pages and fits the device.
  * ODA_OK, or ODA_ERR_INVALID_ARG for another value. */
 int oda_debug_set_local_shape(int index);
 

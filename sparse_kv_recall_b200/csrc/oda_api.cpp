@@ -27,7 +27,7 @@ extern "C" int oda_debug_set_wait_limit(unsigned long long ns) {
 }
 
 extern "C" int oda_debug_set_local_shape(int index) {
-  if (index < -1 || index > 2) return ODA_ERR_INVALID_ARG;
+  if (index < -1 || index > 3) return ODA_ERR_INVALID_ARG;
   oda::g_local_shape.store(index, std::memory_order_relaxed);
   return ODA_OK;
 }

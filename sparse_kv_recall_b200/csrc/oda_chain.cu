@@ -51,8 +51,8 @@ constexpr int kChainMaxHl = 64;       // h^L rows per CTA: 128 G / C, rounded up
 // warps, one page per warp, so C x W pages per (sequence, KV head) at most. The 16 x 9 shape
 // runs two CTAs per SM; the shorter clusters run one CTA per SM (their shared memory is
 // padded to make sure), so that no cluster's page steps and merges share an SM's issue slots.
-constexpr int kChainBufBytesMax = 16 * kStageBytes;
-constexpr int kChainMaxW = 16;
+// The 8 x 18 shape (576 threads, so at most 112 registers a thread) serves one and two query
+// heads per KV head only.
 
 // Floats of the in-CTA merge scratch: the warps' softmax states of G heads (max, sum, 128
 // accumulators each).
@@ -465,13 +465,13 @@ __global__ void __launch_bounds__(W * 32, (C == 16 && G != 4) ? 2 : 1)
         dead = true;
       }
       if (!last && tid == 0) mbar_arrive_expect_tx(ibar, (uint32_t)C * slot_bytes);  // next layer
-      // The merge of the 16 CTA partials, in rank order: one thread per (head, partial)
+      // The merge of the C CTA partials, in rank order: one thread per (head, partial)
       // weighs it against the head's maximum, then one thread per (head, dim) sums.
-      float* wsm = scratch;                 // [G][16] weights (the CTA merge is done with it)
-      float* msm = scratch + 16 * G;        // [G] maxima
+      float* wsm = scratch;                 // [G][C] weights (the CTA merge is done with it)
+      float* msm = scratch + C * G;         // [G] maxima
       constexpr int kOut = ClusterPart<G>::kOut;
-      if (tid < 16 * G) {
-        const int gg = tid / 16, cc = tid % 16;
+      if (tid < C * G) {
+        const int gg = tid / C, cc = tid % C;
         float M = -INFINITY;
 #pragma unroll
         for (int c2 = 0; c2 < C; ++c2) M = fmaxf(M, inbox[c2 * stride + kOut + gg]);
@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(W * 32, (C == 16 && G != 4) ? 2 : 1)
           float Ls = 0.f;
 #pragma unroll
           for (int cc = 0; cc < C; ++cc) {
-            const float wc = wsm[gg * 16 + cc];
+            const float wc = wsm[gg * C + cc];
             const float4 av = *reinterpret_cast<const float4*>(inbox + cc * stride + o);
             Ls += wc;
             ov[0] = fmaf(wc, av.x, ov[0]);
@@ -720,15 +720,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) full_chain_kernel(const 
 struct ChainShape {
   int C, W;
 };
-constexpr ChainShape kChainShapes[] = {{16, 9}, {14, 10}, {12, 11}};
-constexpr int kNumChainShapes = 3;
+constexpr ChainShape kChainShapes[] = {{16, 9}, {14, 10}, {12, 11}, {8, 18}};
+constexpr int kNumChainShapes = 4;
+// Shapes tried in this order (the first whose clusters are all resident at once is used).
+constexpr int kChainPrefer[kNumChainShapes] = {3, 1, 2, 0};
 
 // Dynamic shared memory of the Local kernel: page buffer, merge scratch, barriers, per-warp
 // softmax exchange, rank 0's inbox; for the one-CTA-per-SM shapes at least kOneCtaSmem.
 constexpr size_t kOneCtaSmem = 118 * 1024;
 static size_t local_chain_smem(int G, ChainShape sh, int inbox_stride) {
-  const int scratch = sh.W == 9 ? chain_scratch_floats<9>(G)
-                    : (sh.W == 10 ? chain_scratch_floats<10>(G) : chain_scratch_floats<11>(G));
+  const int scratch = sh.W == 9    ? chain_scratch_floats<9>(G)
+                      : sh.W == 10 ? chain_scratch_floats<10>(G)
+                      : sh.W == 11 ? chain_scratch_floats<11>(G)
+                                   : chain_scratch_floats<18>(G);
   size_t n = (size_t)sh.W * kStageBytes + (size_t)scratch * sizeof(float) +
              (sh.W + 3) * sizeof(uint64_t) + (size_t)sh.W * 18 * G * sizeof(float) + 16 +
              (size_t)(sh.C + 1) * inbox_stride * sizeof(float);
@@ -822,9 +826,16 @@ static cudaError_t local_attrs(int optin, int* max_dyn) {
 
 // The instances by (group size, shape index): one dispatch per operation.
 #define ODA_LOCAL_INSTANCES(X) \
-  X(1, 0, 16, 9) X(1, 1, 14, 10) X(1, 2, 12, 11) \
-  X(2, 0, 16, 9) X(2, 1, 14, 10) X(2, 2, 12, 11) \
+  X(1, 0, 16, 9) X(1, 1, 14, 10) X(1, 2, 12, 11) X(1, 3, 8, 18) \
+  X(2, 0, 16, 9) X(2, 1, 14, 10) X(2, 2, 12, 11) X(2, 3, 8, 18) \
   X(4, 0, 16, 9) X(4, 1, 14, 10) X(4, 2, 12, 11)
+static bool local_has(int G, int si) {
+#define ODA_X(g, i, c, w) \
+  if (G == g && si == i) return true;
+  ODA_LOCAL_INSTANCES(ODA_X)
+#undef ODA_X
+  return false;
+}
 
 static cudaError_t local_launch(int G, int si, const LocalChainParams& p, int clusters,
                                 size_t smem, cudaStream_t st, bool coop) {
@@ -879,7 +890,7 @@ int prepare_chain_kernels() {
   if (e != cudaSuccess) return cuda_status(e);
   for (int G : {1, 2, 4})
     for (int si = 0; si < kNumChainShapes; ++si)
-      if ((e = local_set_attrs(G, si, optin, &f.max_dyn[G][si])) != cudaSuccess)
+      if (local_has(G, si) && (e = local_set_attrs(G, si, optin, &f.max_dyn[G][si])) != cudaSuccess)
         return cuda_status(e);
   if ((rc = prepare_full_g<1>(f)) != ODA_OK) return rc;
   if ((rc = prepare_full_g<2>(f)) != ODA_OK) return rc;
@@ -950,7 +961,7 @@ static bool recall_fusable(const oda_step_desc* d, int B, int G, ChainShape sh, 
 
 int plan_local_chain(const oda_step_desc* d, int phases, LocalChainPlan* pl) {
   *pl = LocalChainPlan{};
-  if (!(phases & ODA_PHASE_LOCAL) || d->step_kernels == ODA_STEP_PER_LAYER) return ODA_OK;
+  if (!(phases & ODA_PHASE_LOCAL) || d->step_kernels != ODA_STEP_PERSISTENT) return ODA_OK;
   DeviceInfo di;
   int rc = current_device_info(&di);
   if (rc != ODA_OK) return rc;
@@ -975,7 +986,7 @@ int plan_local_chain(const oda_step_desc* d, int phases, LocalChainPlan* pl) {
   // shapes in order of preference (one CTA per SM first), or the one a tuning hook names
   const int forced = test_local_shape();
   for (int k = 0; k < kNumChainShapes; ++k) {
-    const int si = forced >= 0 ? forced : (k + 1) % kNumChainShapes;
+    const int si = forced >= 0 ? forced : kChainPrefer[k];
     if (forced >= 0 && k > 0) break;
     const ChainShape sh = kChainShapes[si];
     if (max_pages > (long long)sh.C * sh.W) continue;

@@ -61,7 +61,7 @@ int layer_window(const oda_step_desc* d, int l) { return d->windows ? d->windows
 int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditionalHandle cond) {
   const int L = d->num_layers;
   const int phases = d->phases ? d->phases : (ODA_PHASE_LOCAL | ODA_PHASE_RECALL | ODA_PHASE_FULL);
-  const bool persistent = d->step_kernels != ODA_STEP_PER_LAYER;
+  const bool persistent = d->step_kernels != ODA_STEP_PER_LAYER;  // (Full; Local: the plan)
   const unsigned long long cond_u64 = d->use_conditional ? (unsigned long long)cond : 0ull;
   int rc;
   if (g->timing && (rc = record_event_node(g, 0)) != ODA_OK) return rc;
@@ -201,7 +201,8 @@ int check_desc(const oda_step_desc* d) {
   if (d->gate_source == ODA_GATE_RANDOM &&
       (d->gate_u == nullptr || !(d->rho >= 0.f && d->rho <= 1.f)))
     return ODA_ERR_INVALID_ARG;
-  if (d->step_kernels != ODA_STEP_PERSISTENT && d->step_kernels != ODA_STEP_PER_LAYER)
+  if (d->step_kernels != ODA_STEP_FULL_PERSISTENT && d->step_kernels != ODA_STEP_PER_LAYER &&
+      d->step_kernels != ODA_STEP_PERSISTENT)
     return ODA_ERR_INVALID_ARG;
   return ODA_OK;
 }

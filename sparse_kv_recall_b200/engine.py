@@ -79,7 +79,7 @@ class OdaEngine:
                  sinks: Optional[Sequence[int]] = None, windows: Optional[Sequence[int]] = None,
                  random_rho: Optional[float] = None,
                  with_lse: bool = False, with_stats: bool = True, phases: int = 0,
-                 step_kernels: int = oda.ODA_STEP_PERSISTENT):
+                 step_kernels: int = oda.ODA_STEP_FULL_PERSISTENT):
         self.L = len(k_caches)
         self.B = block_table.shape[0]
         self.hq = num_q_heads

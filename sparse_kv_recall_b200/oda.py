@@ -43,8 +43,9 @@ ODA_PHASE_RECALL = 2
 ODA_PHASE_FULL = 4
 ODA_GATE_RECALL = 0
 ODA_GATE_RANDOM = 1
-ODA_STEP_PERSISTENT = 0
+ODA_STEP_FULL_PERSISTENT = 0
 ODA_STEP_PER_LAYER = 1
+ODA_STEP_PERSISTENT = 2
 ODA_STALL_NONE = 0
 ODA_STALL_DECODE_RING = 1
 ODA_STALL_LOCAL_CHAIN = 2
@@ -383,7 +384,7 @@ class StepGraph:
                  decode_ws, recall_ws, full_count=None, lse=None, local_layers=None,
                  sinks=None, windows=None, use_conditional: bool = True,
                  timing_events: bool = False, phases: int = 0, gate_u=None, rho: float = 0.0,
-                 step_kernels: int = ODA_STEP_PERSISTENT):
+                 step_kernels: int = ODA_STEP_FULL_PERSISTENT):
         L = len(kvs)
         self._keep = []
         layers = (oda_kv * L)(*kvs)

@@ -31,7 +31,7 @@ def _logical(bits, bt, caps, hkv, d):
 
 
 def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02, timing=False,
-               step_kernels=oda.ODA_STEP_PERSISTENT, expect_kernels=None, **layer_ranges):
+               step_kernels=oda.ODA_STEP_FULL_PERSISTENT, expect_kernels=None, **layer_ranges):
     lay = oda_synth.make_layout(w, extra_tokens=steps + 2, device="cuda", lengths=lengths)
     caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
     rw = oda_synth.make_recall_weights(w, device="cuda", std=recall_std)
@@ -186,6 +186,7 @@ def test_local_only_phase_graph():
 
 # ---- the persistent step kernels: Local at every layer + fused gate as one launch (one
 # cluster per (sequence, KV head), batch x KV heads <= 9 clusters), Full as one launch ----
+P = oda.ODA_STEP_PERSISTENT
 
 def _expected_kernels(w):
     """(Local, gate, Full) launches per step the step graph should take on this device: the
@@ -194,7 +195,8 @@ def _expected_kernels(w):
     G, ncl = w.num_q_heads // w.num_kv_heads, w.batch * w.num_kv_heads
     fused, _ = oda.oda_step_kernel_limits(G, w.batch, w.mlp)
     plain, _ = oda.oda_step_kernel_limits(G, w.batch, 0)
-    if fused >= ncl:
+    slabs = -(-3 * w.num_q_heads * 128 // 256)              # the recall head's row slabs
+    if fused >= ncl and ncl <= slabs:
         return (1, 0, 1)
     if plain >= ncl:
         return (1, 1, 1)
@@ -222,7 +224,7 @@ def test_persistent_step_kernels_match_oracle(use_conditional, hq, hkv, batch, l
                            num_kv_heads=hkv, prefill=max(lengths), steps=5, seed=90 + hq + batch,
                            sink=4, window=128)
     n = _run_steps(w, lengths, 5, theta=0.0, use_conditional=use_conditional,
-                   expect_kernels=_expected_kernels(w))
+                   step_kernels=P, expect_kernels=_expected_kernels(w))
     assert 0 < n < 5 * batch
 
 
@@ -230,21 +232,23 @@ def test_persistent_step_kernels_per_layer_sink_and_window():
     w = oda_synth.Workload(name="chain-ranges", layers=3, batch=1, num_q_heads=16,
                            num_kv_heads=8, prefill=900, steps=4, seed=93, sink=4, window=64)
     _run_steps(w, [900], 4, theta=0.0, sinks=[4, 0, 16], windows=[64, 17, 2000],
-               expect_kernels=(1, 0, 1))
+               step_kernels=P, expect_kernels=(1, 0, 1))
 
 
 def test_persistent_step_kernels_random_schedule_and_ends():
     w = oda_synth.Workload(name="chain-random", layers=2, batch=1, num_q_heads=16,
                            num_kv_heads=8, prefill=400, steps=6, seed=94, sink=4, window=64)
-    _run_steps(w, [400], 6, theta=0.0, random_rho=0.5, expect_kernels=(1, 0, 1))
-    assert _run_steps(w, [400], 3, theta=float("inf"), expect_kernels=(1, 0, 1)) == 0
-    assert _run_steps(w, [400], 3, theta=-float("inf"), expect_kernels=(1, 0, 1)) == 3
+    _run_steps(w, [400], 6, theta=0.0, random_rho=0.5, step_kernels=P, expect_kernels=(1, 0, 1))
+    assert _run_steps(w, [400], 3, theta=float("inf"), step_kernels=P,
+                      expect_kernels=(1, 0, 1)) == 0
+    assert _run_steps(w, [400], 3, theta=-float("inf"), step_kernels=P,
+                      expect_kernels=(1, 0, 1)) == 3
 
 
 def test_persistent_step_kernels_with_timing_events():
     w = oda_synth.Workload(name="chain-timing", layers=2, batch=1, num_q_heads=16,
                            num_kv_heads=8, prefill=600, steps=3, seed=95, sink=4, window=256)
-    _run_steps(w, [600], 3, theta=0.0, timing=True, expect_kernels=(1, 0, 1))
+    _run_steps(w, [600], 3, theta=0.0, timing=True, step_kernels=P, expect_kernels=(1, 0, 1))
 
 
 def test_shapes_outside_the_persistent_local_kernel_fall_back():
@@ -252,7 +256,7 @@ def test_shapes_outside_the_persistent_local_kernel_fall_back():
     layer with the recall kernel after it, Full still as one persistent launch."""
     w = oda_synth.Workload(name="chain-fallback", layers=2, batch=3, num_q_heads=16,
                            num_kv_heads=8, prefill=300, steps=3, seed=96, sink=4, window=64)
-    _run_steps(w, [300, 37, 170], 3, theta=0.0, expect_kernels=(2, 1, 1))
+    _run_steps(w, [300, 37, 170], 3, theta=0.0, step_kernels=P, expect_kernels=(2, 1, 1))
 
 
 @pytest.mark.parametrize("theta", [float("inf"), -float("inf")])
@@ -261,13 +265,14 @@ def test_persistent_step_equals_per_layer(theta):
     recomputed by Full (theta = -inf) every layer output is bitwise the per-layer launches'.
     The persistent Local kernel forms its page scores on the tensor cores and merges one state
     per warp (the per-layer cluster kernel: CUDA-core scores, two states per warp), so Local
-    outputs (theta = +inf) agree to fp32 rounding. Committed K/V bits and the attended-row and
-    page counters are identical either way; theta at +-inf keeps the gate out of it (the fused
-    recall head sums in another order than the recall kernel)."""
+    outputs (theta = +inf) agree to fp32 rounding. The default mode (Local per layer, Full
+    persistent) equals the per-layer launches bitwise at both ends. Committed K/V bits and the
+    attended-row and page counters are identical either way; theta at +-inf keeps the gate out
+    of it (the fused recall head sums in another order than the recall kernel)."""
     w = oda_synth.Workload(name="chain-bitwise", layers=3, batch=1, num_q_heads=16,
                            num_kv_heads=8, prefill=3000, steps=3, seed=97, sink=4, window=512)
     res = {}
-    for sk in (oda.ODA_STEP_PERSISTENT, oda.ODA_STEP_PER_LAYER):
+    for sk in (oda.ODA_STEP_PERSISTENT, oda.ODA_STEP_PER_LAYER, oda.ODA_STEP_FULL_PERSISTENT):
         lay = oda_synth.make_layout(w, extra_tokens=5, device="cuda")
         caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
         rw = oda_synth.make_recall_weights(w, device="cuda")
@@ -294,3 +299,32 @@ def test_persistent_step_equals_per_layer(theta):
     for (ka, va), (kb, vb) in zip(a[1], b[1]):
         assert torch.equal(ka, kb) and torch.equal(va, vb)
     assert torch.equal(a[2], b[2])                       # rows / pages counters
+    c = res[oda.ODA_STEP_FULL_PERSISTENT]
+    assert torch.equal(c[0], b[0]) and torch.equal(c[2], b[2])
+    for (kc, vc), (kb, vb) in zip(c[1], b[1]):
+        assert torch.equal(kc, kb) and torch.equal(vc, vb)
+
+
+@pytest.mark.parametrize("shape", [0, 1, 2, 3])
+@pytest.mark.parametrize("hq,hkv,batch,lengths", [
+    (8, 4, 1, [900]),            # two query heads per KV head
+    (4, 2, 2, [700, 60]),        # inbox slots sized by the fused recall head (batch x mlp)
+    (4, 4, 1, [500]),            # one query head per KV head
+    (16, 4, 1, [400]),           # four query heads per KV head (no 8 x 18 instance)
+])
+def test_persistent_local_every_shape_matches_oracle(shape, hq, hkv, batch, lengths):
+    """Each cluster shape of the persistent Local kernel (16 x 9, 14 x 10, 12 x 11, 8 x 18 CTAs
+    x warps), forced through the tuning hook, with the fused recall head, against the oracle.
+    Four clusters or fewer fit every shape; a group size a shape has no instance of falls back
+    to one launch per layer."""
+    w = oda_synth.Workload(name="chain-shape", layers=2, batch=batch, num_q_heads=hq,
+                           num_kv_heads=hkv, prefill=max(lengths), steps=3,
+                           seed=300 + 10 * shape + hq + batch, sink=4, window=128)
+    G = hq // hkv
+    expect = (w.layers, 1, 1) if (G == 4 and shape == 3) else (1, 0, 1)
+    oda.oda_debug_set_local_shape(shape)
+    try:
+        _run_steps(w, lengths, 3, theta=0.0, use_conditional=False, step_kernels=P,
+                   expect_kernels=expect)
+    finally:
+        oda.oda_debug_set_local_shape(-1)

@@ -43,7 +43,10 @@ class _Stall:
 def test_hooks_reject_unknown_kinds():
     with pytest.raises(oda.OdaError, match="INVALID_ARG"):
         oda.oda_debug_set_stall(17)
+    with pytest.raises(oda.OdaError, match="INVALID_ARG"):
+        oda.oda_debug_set_local_shape(4)
     oda.oda_debug_set_stall(oda.ODA_STALL_NONE)
+    oda.oda_debug_set_local_shape(-1)
 
 
 def test_decode_ring_wait_runs_out_then_recovers():
@@ -64,13 +67,13 @@ def test_decode_ring_wait_runs_out_then_recovers():
     assert_lse_close(lse.cpu().numpy(), rlse)
 
 
-def _engine(w, lengths, theta, **kw):
+def _engine(w, lengths, theta, step_kernels=oda.ODA_STEP_PERSISTENT, **kw):
     lay = oda_synth.make_layout(w, extra_tokens=8, device="cuda", lengths=lengths)
     caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
     rw = oda_synth.make_recall_weights(w, device="cuda")
     eng = OdaEngine([c[0] for c in caches], [c[1] for c in caches], lay.block_table,
                     w.num_q_heads, (rw.w1, rw.b1, rw.w2, rw.b2), theta, sink=w.sink,
-                    window=w.window, use_conditional=False, **kw)
+                    window=w.window, use_conditional=False, step_kernels=step_kernels, **kw)
     h0 = oda_synth.make_h0(w, device="cuda")
     eng.set_h_prev(h0, 0)
     return eng, lay, caches, rw, h0
