@@ -333,6 +333,31 @@ def test_repeat_runs_are_bitwise_identical():
     assert torch.equal(a, b) and torch.equal(la, lb)
 
 
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_long_segments_are_bitwise_repeatable_and_match_oracle(G):
+    """Repeated launches over long and short segments (a 128K one spread over every CTA of the
+    grid, one across share boundaries, short ones) agree bit for bit -- each partial is formed
+    and merged in a fixed order -- and match the oracle; the launch-wide counters in the
+    workspace stay zero."""
+    lens = [131_073, 8_192 + 17, 8_191, 300, 1]
+    c = Case(lens, hq=8 * G, hkv=8, seed=140 + G)
+    outs = []
+    for _ in range(3):
+        out, lse = c.out_buffers()
+        _run(c, lambda: oda.oda_decode_full(c.kv, c.q, SCALE, out, c.ws, lse=lse))
+        outs.append((out, lse))
+    for out, lse in outs[1:]:
+        assert torch.equal(out, outs[0][0]) and torch.equal(lse, outs[0][1])
+    ref, rlse = c.oracle(lambda b, t: O.full_positions(t))
+    assert_attn_close(outs[0][0].cpu().numpy(), ref, "full over long segments G=%d" % G)
+    assert_lse_close(outs[0][1].cpu().numpy(), rlse)
+    st = c.stats.cpu().numpy()
+    assert st[oda.ODA_STAT_ROWS] == 3 * 8 * sum(lens)                 # every row once per launch
+    assert st[oda.ODA_STAT_PAGES] == 3 * 8 * sum((n + 15) // 16 for n in lens)
+    ws_tail = c.ws.view(torch.int32)[-64:]
+    assert int(ws_tail.abs().sum().item()) == 0                       # counters left zero
+
+
 def test_bf16_output_within_one_ulp():
     c = Case([700, 3333], hq=16, hkv=8, seed=91)
     out, _ = c.out_buffers(dtype=torch.bfloat16)

@@ -259,8 +259,9 @@ def test_shapes_outside_the_persistent_local_kernel_fall_back():
     _run_steps(w, [300, 37, 170], 3, theta=0.0, step_kernels=P, expect_kernels=(2, 1, 1))
 
 
-@pytest.mark.parametrize("theta", [float("inf"), -float("inf")])
-def test_persistent_step_equals_per_layer(theta):
+@pytest.mark.parametrize("theta,prefill", [(float("inf"), 3000), (-float("inf"), 3000),
+                                           (-float("inf"), 9000)])
+def test_persistent_step_equals_per_layer(theta, prefill):
     """The persistent Full kernel runs the per-layer split pass itself, so with every step
     recomputed by Full (theta = -inf) every layer output is bitwise the per-layer launches'.
     The persistent Local kernel forms its page scores on the tensor cores and merges one state
@@ -268,9 +269,10 @@ def test_persistent_step_equals_per_layer(theta):
     outputs (theta = +inf) agree to fp32 rounding. The default mode (Local per layer, Full
     persistent) equals the per-layer launches bitwise at both ends. Committed K/V bits and the
     attended-row and page counters are identical either way; theta at +-inf keeps the gate out
-    of it (the fused recall head sums in another order than the recall kernel)."""
+    of it (the fused recall head sums in another order than the recall kernel). The 9000-token
+    case spreads each segment over many CTAs of the grid."""
     w = oda_synth.Workload(name="chain-bitwise", layers=3, batch=1, num_q_heads=16,
-                           num_kv_heads=8, prefill=3000, steps=3, seed=97, sink=4, window=512)
+                           num_kv_heads=8, prefill=prefill, steps=3, seed=97, sink=4, window=512)
     res = {}
     for sk in (oda.ODA_STEP_PERSISTENT, oda.ODA_STEP_PER_LAYER, oda.ODA_STEP_FULL_PERSISTENT):
         lay = oda_synth.make_layout(w, extra_tokens=5, device="cuda")
