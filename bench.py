@@ -45,10 +45,24 @@ FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0         # B200 HBM3e nominal (~8 TB/s), reported beside the measured peak
 # Machine-readable ncu figures (written by `bench.py --ncu-summary` from a capture's raw CSV),
 # beside the prose summaries of the same captures in profiles/*.md.
-PROFILE = os.path.join(ROOT, "profiles", "full_chain_128k.json")
-LOCAL_PROFILE = os.path.join(ROOT, "profiles", "local_chain_128k.json")
+# Committed ncu summaries (JSON written by --ncu-summary) of the step's kernels on the
+# long-context workload, by kernel, and the device sources each was taken on.
+PROFILES = {
+    "full_chain": os.path.join(ROOT, "profiles", "full_chain_128k.json"),
+    "full_layer": os.path.join(ROOT, "profiles", "decode_full_128k.json"),
+    "local_cluster": os.path.join(ROOT, "profiles", "local_cluster_128k.json"),
+    "local_chain": os.path.join(ROOT, "profiles", "local_chain_128k.json"),
+    "recall": os.path.join(ROOT, "profiles", "recall_h2048.json"),
+}
+PROFILE = PROFILES["full_chain"]
 KERNEL_SOURCES = ["oda_decode.cuh", "oda_decode.cu", "oda_chain.cu", "oda_plan.cuh",
                   "oda_common.cuh", "oda_recall.cuh"]
+RECALL_SOURCES = ["oda_recall.cu", "oda_recall.cuh", "oda_common.cuh"]
+
+
+def profile_sources(key_or_kernel: str):
+    """Device sources an ncu summary of this kernel depends on."""
+    return RECALL_SOURCES if "recall" in key_or_kernel else KERNEL_SOURCES
 
 
 STEP_KERNELS = {"full-persistent": 0, "per-layer": 1, "persistent": 2}  # ODA_STEP_*
@@ -232,11 +246,12 @@ def _profile_fields(path: str, sources=None) -> dict:
     return info if info.get("source_sha") == kernel_source_hash(sources) else {}
 
 
-def profiled_traffic(n_ctx_tokens_per_layer: float, layers: int = 1):
+def profiled_traffic(n_ctx_tokens_per_layer: float, layers: int = 1, key: str = "full_chain"):
     """DRAM bytes of a Full launch covering `layers` layers at this many context tokens per
-    layer, from the committed ncu capture of the persistent Full kernel (scaled by tokens and
-    layers, as its traffic grows in proportion); None when missing or stale."""
-    info = _profile_fields(PROFILE)
+    layer, from the committed ncu capture of that Full kernel (the persistent one, or one
+    layer of the split kernel), scaled by tokens and layers, as its traffic grows in
+    proportion; None when missing or stale."""
+    info = _profile_fields(PROFILES[key], profile_sources(key))
     try:
         per_token = float(info["dram_bytes_per_launch"]) / (
             float(info["tokens_per_layer"]) * float(info["layers_per_launch"]))
@@ -245,17 +260,26 @@ def profiled_traffic(n_ctx_tokens_per_layer: float, layers: int = 1):
         return None
 
 
-def profiled_step_bytes(layers: int, full_phases_per_step: float, n_ctx_tokens: float):
-    """DRAM bytes one step of the default workload reads and writes, from the committed ncu
-    captures of its kernels (the persistent Local kernel with the fused recall head, the
-    persistent Full kernel on the steps that run it): the "bytes actually read" figure beside
-    the attended (algorithmic) bytes. None when any capture is missing or stale."""
+def profiled_step_bytes(mode: str, layers: int, full_phases_per_step: float,
+                        n_ctx_tokens: float):
+    """DRAM bytes one step of the long-context workload reads and writes, from the committed
+    ncu captures of the kernels the step mode runs (Local: the per-layer cluster kernel and
+    the recall kernel, or the persistent Local kernel with the fused recall head; Full: the
+    persistent Full kernel, or one split launch per layer, on the steps that run it): the
+    "bytes actually moved" figure beside the attended (algorithmic) bytes. None when a capture
+    is missing or stale."""
+    def per_launch(key):
+        info = _profile_fields(PROFILES[key], profile_sources(key))
+        return float(info["dram_bytes_per_launch"]) / float(info.get("layers_per_launch", 1))
     try:
-        loc = _profile_fields(LOCAL_PROFILE)
-        local = float(loc["dram_bytes_per_launch"]) * layers / float(loc["layers_per_launch"])
+        if mode == "persistent":
+            local = per_launch("local_chain") * layers
+        else:
+            local = per_launch("local_cluster") * layers + per_launch("recall")
     except (KeyError, ValueError, ZeroDivisionError):
         return None
-    full = profiled_traffic(n_ctx_tokens, layers)
+    full = profiled_traffic(n_ctx_tokens, layers,
+                            "full_layer" if mode == "per-layer" else "full_chain")
     if full is None:
         return None
     return local + full_phases_per_step * full
@@ -293,7 +317,7 @@ def ncu_summary(csv_path: str, kernel: str, out_path: str, extra: dict) -> dict:
 
     info = dict(extra)
     info.update({"kernel": picked[0][ki][:120], "launches_captured": len(picked),
-                 "source_sha": kernel_source_hash(),
+                 "source_sha": kernel_source_hash(profile_sources(kernel)),
                  "dram_bytes_read_per_launch": mean("dram__bytes_read.sum"),
                  "dram_bytes_write_per_launch": mean("dram__bytes_write.sum")})
     info["dram_bytes_per_launch"] = (info["dram_bytes_read_per_launch"]
@@ -929,7 +953,7 @@ def run_oda(args, dist: Dist):
         # DRAM bytes of the step's kernels as ncu counted them (committed summaries), with the
         # Full launches at the timed region's mean context
         ctx_mid = float(np.mean(s.lengths)) + step0 + K / 2.0 + 1.0
-        sb = profiled_step_bytes(w.layers, fc[1] / float(K), ctx_mid * w.batch)
+        sb = profiled_step_bytes(args.step_kernels, w.layers, fc[1] / float(K), ctx_mid * w.batch)
         result["kv_stream"]["ncu_bytes_per_step"] = sb
         result["kv_stream"]["ncu_gbs"] = (sb * K / (ms_local / 1e3) / 1e9) if sb else None
         result["kv_stream"]["ncu_frac_of_peak"] = (sb * K / (ms_local / 1e3) / 1e9 / peak
@@ -998,7 +1022,8 @@ def run_oda(args, dist: Dist):
     else:
         achieved, alg, ms_launch, how = achieved_alone, alg_layer, dur, "one layer alone"
     traffic = profiled_traffic(alg / (w.num_kv_heads * ROW_BYTES * w.layers), w.layers) \
-        if full_launches == 1 else profiled_traffic(alg / (w.num_kv_heads * ROW_BYTES), 1)
+        if full_launches == 1 else profiled_traffic(alg / (w.num_kv_heads * ROW_BYTES), 1,
+                                                    "full_layer")
     name = ("full_chain_kernel<%d> (Full at every layer, one launch)" % w.group
             if full_launches == 1 else "decode_kernel<%d> (Full, one layer)" % w.group)
     result["roofline"] = {"kernel": name,

@@ -72,8 +72,8 @@ def test_clock_sampler_without_nvidia_smi_is_reported():
 
 def test_profiled_bytes_follow_committed_captures(tmp_path, monkeypatch):
     """bench.py reads the DRAM bytes of the step's kernels from the JSON its --ncu-summary
-    writes from an ncu capture, and only while the kernel sources it was taken on are
-    unchanged; the summary is read back from a raw CSV export the way ncu writes it."""
+    writes from an ncu capture, by step mode, and only while the kernel sources it was taken
+    on are unchanged; the summary is read back from a raw CSV export the way ncu writes it."""
     import bench
     csv = tmp_path / "raw.csv"
     csv.write_text(
@@ -82,23 +82,38 @@ def test_profiled_bytes_follow_committed_captures(tmp_path, monkeypatch):
         '"","","","Mbyte","Mbyte","usecond"\n'
         '"0","1","void oda::local_chain_kernel<2>(oda::LocalChainParams)","200.5","1.5","40"\n'
         '"1","1","void oda::full_chain_kernel<2>(oda::FullChainParams)","1,080","8","200"\n'
-        '"2","1","void oda::full_chain_kernel<2>(oda::FullChainParams)","1,082","8","202"\n')
-    full = tmp_path / "full.json"
-    info = bench.ncu_summary(str(csv), "full_chain_kernel", str(full),
+        '"2","1","void oda::full_chain_kernel<2>(oda::FullChainParams)","1,082","8","202"\n'
+        '"3","1","void oda::cluster_decode_kernel<2>(oda::DecodeParams)","8.5","0.5","6"\n'
+        '"4","1","void oda::recall_kernel(oda::RecallParams)","6.3","0.1","4"\n')
+    paths = {k: tmp_path / (k + ".json") for k in bench.PROFILES}
+    info = bench.ncu_summary(str(csv), "full_chain_kernel", str(paths["full_chain"]),
                              {"tokens_per_layer": 131073, "layers_per_launch": 2})
     assert info["launches_captured"] == 2
     assert info["dram_bytes_per_launch"] == 1089e6
     assert abs(info["gpu_time_s_per_launch_under_ncu"] - 201e-6) < 1e-12
-    local = tmp_path / "local.json"
-    bench.ncu_summary(str(csv), "local_chain_kernel", str(local), {"layers_per_launch": 28})
-    monkeypatch.setattr(bench, "PROFILE", str(full))
-    monkeypatch.setattr(bench, "LOCAL_PROFILE", str(local))
+    bench.ncu_summary(str(csv), "local_chain_kernel", str(paths["local_chain"]),
+                      {"layers_per_launch": 28})
+    bench.ncu_summary(str(csv), "cluster_decode_kernel", str(paths["local_cluster"]),
+                      {"layers_per_launch": 1})
+    bench.ncu_summary(str(csv), "recall_kernel", str(paths["recall"]), {})
+    monkeypatch.setattr(bench, "PROFILES", {k: str(v) for k, v in paths.items()})
     per = 1089e6 / (131073 * 2)
     assert abs(bench.profiled_traffic(131073, 28) - per * 131073 * 28) < 1.0
-    step = bench.profiled_step_bytes(28, 0.5, 131073)
-    assert abs(step - (202e6 + 0.5 * per * 131073 * 28)) < 1.0
-    stale = json.load(open(full))
+    step = bench.profiled_step_bytes("persistent", 28, 0.5, 131073)
+    assert abs(step - (202e6 * 28 / 28 + 0.5 * per * 131073 * 28)) < 1.0
+    step = bench.profiled_step_bytes("full-persistent", 28, 0.5, 131073)
+    assert abs(step - (9e6 * 28 + 6.4e6 + 0.5 * per * 131073 * 28)) < 1.0
+    assert bench.profiled_step_bytes("per-layer", 28, 0.5, 131073) is None   # no capture
+    stale = json.load(open(paths["full_chain"]))
     stale["source_sha"] = "0000000000000000"
-    json.dump(stale, open(full, "w"))
+    json.dump(stale, open(paths["full_chain"], "w"))
     assert bench.profiled_traffic(131073, 28) is None
-    assert bench.profiled_step_bytes(28, 0.5, 131073) is None
+    assert bench.profiled_step_bytes("full-persistent", 28, 0.5, 131073) is None
+
+
+def test_bench_step_kernel_modes_match_the_library():
+    import bench
+    from sparse_kv_recall_b200 import oda
+    assert bench.STEP_KERNELS == {"full-persistent": oda.ODA_STEP_FULL_PERSISTENT,
+                                  "per-layer": oda.ODA_STEP_PER_LAYER,
+                                  "persistent": oda.ODA_STEP_PERSISTENT}
