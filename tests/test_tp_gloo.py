@@ -136,7 +136,7 @@ def _worker(rank, world, port, out):
 
 @pytest.mark.parametrize("world", [2, 4])
 def test_head_parallel_steps_equal_the_oracle_step(world):
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     for rank in range(world):
         err, gates_equal, gate_match, commits, _ = out[rank]
