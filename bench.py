@@ -350,7 +350,7 @@ class Setup:
         self.eng = OdaEngine([c[0] for c in self.caches], [c[1] for c in self.caches],
                              self.layout.block_table, w.num_q_heads, self.recall, theta,
                              sink=w.sink, window=w.window, use_conditional=use_conditional,
-                             step_kernels=step_kernels)
+                             step_kernels=step_kernels, staging_slots=2)
         self.eng.set_h_prev(oda_synth.make_h0(w, device=dev), 0)
         lay = StagingLayout(w.layers, w.batch, w.num_q_heads, w.num_kv_heads, w.hidden)
         self.slot = lay.nbytes
@@ -361,7 +361,8 @@ class Setup:
         torch.cuda.synchronize()
 
     def feed(self, i: int):
-        self.eng.staging.copy_(self.pool[i], non_blocking=True)
+        """Step i's inputs from the resident pool into the staging slot its graph reads."""
+        self.eng.staging_for(i).copy_(self.pool[i], non_blocking=True)
 
 
 def launches_per_step(kernels, phases: int, steps: int, conditional: bool = True) -> int:
@@ -1046,26 +1047,55 @@ def run_oda(args, dist: Dist):
         host_pool = torch.empty((E2E, s.slot), dtype=torch.uint8, pin_memory=True)
         host_pool.copy_(s.pool[step:step + E2E])
         out_h = torch.empty((2, w.batch, w.hidden), dtype=torch.float32, pin_memory=True)
-        gate_h = torch.empty((2, w.batch), dtype=torch.int32, pin_memory=True)
         torch.cuda.synchronize()
         dist.barrier()
         fc_e = eng.full_count.clone()
+        # Two staging slots: step i's inputs go in on an input stream while step i - 1 runs,
+        # once the graph of step i - 2 (same slot) has finished; step i's selected output (its
+        # result) comes back on an output stream while step i + 1 runs, before step i + 2
+        # overwrites it. (One stream for both would queue step i + 1's inputs behind step i's
+        # output read, which waits for step i to finish.)
+        cs_in, cs_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ran = [torch.cuda.Event() for _ in range(2)]      # step graph of this slot finished
+        staged = [torch.cuda.Event() for _ in range(2)]   # inputs of this slot copied in
+        read = [torch.cuda.Event() for _ in range(2)]     # outputs of this slot copied out
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
+        cs_in.wait_stream(stream)
+        cs_out.wait_stream(stream)
         for i in range(E2E):
-            eng.staging.copy_(host_pool[i], non_blocking=True)
-            eng.launch(step)
-            out_h[i % 2].copy_(eng.selected_last(step), non_blocking=True)
-            gate_h[i % 2].copy_(eng.gate, non_blocking=True)
+            k = step % 2
+            if i >= 2:
+                cs_in.wait_event(ran[k])
+            with torch.cuda.stream(cs_in):
+                eng.staging_for(step).copy_(host_pool[i], non_blocking=True)
+            staged[k].record(cs_in)
+            stream.wait_event(staged[k])
+            if i >= 2:
+                stream.wait_event(read[k])
+            eng.launch(step, stream)
+            ran[k].record(stream)
+            cs_out.wait_event(ran[k])
+            with torch.cuda.stream(cs_out):
+                out_h[i % 2].copy_(eng.selected_last(step), non_blocking=True)
+            read[k].record(cs_out)
             step += 1
+        stream.wait_stream(cs_in)
+        stream.wait_stream(cs_out)
         b.record(stream)
         torch.cuda.synchronize()
         dist.barrier()
         ms_e2e = dist.max(a.elapsed_time(b))
+        rho_e = float((eng.full_count - fc_e)[0].item()) / (w.batch * E2E)
+        gc = result.get("gate_cost", {}).get("ms_per_step", {})
+        dev_model = (gc["theta_plus_inf"] + rho_e * (gc["theta_minus_inf"] - gc["theta_plus_inf"])
+                     if gc else None)
         result["e2e"] = {"value": dist.sum(w.batch * E2E) / (ms_e2e / 1e3), "unit": UNIT,
                          "h2d_bytes_per_step": s.slot,
-                         "d2h_bytes_per_step": w.batch * (w.hidden * 4 + 4), "steps": E2E,
-                         "rho_realised": float((eng.full_count - fc_e)[0].item()) / (w.batch * E2E),
+                         "d2h_bytes_per_step": w.batch * w.hidden * 4, "steps": E2E,
+                         "ms_per_step": ms_e2e / E2E,
+                         "device_ms_per_step_at_its_rho": dev_model,
+                         "rho_realised": rho_e,
                          "note": "its own steps (later in the same decode), so its Full-call "
                                  "rate differs from the main region's"}
     assert int(eng.status.item()) == 0, "device status %d" % int(eng.status.item())

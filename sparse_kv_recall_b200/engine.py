@@ -79,7 +79,7 @@ class OdaEngine:
                  sinks: Optional[Sequence[int]] = None, windows: Optional[Sequence[int]] = None,
                  random_rho: Optional[float] = None,
                  with_lse: bool = False, with_stats: bool = True, phases: int = 0,
-                 step_kernels: int = oda.ODA_STEP_FULL_PERSISTENT):
+                 step_kernels: int = oda.ODA_STEP_FULL_PERSISTENT, staging_slots: int = 1):
         self.L = len(k_caches)
         self.B = block_table.shape[0]
         self.hq = num_q_heads
@@ -96,13 +96,22 @@ class OdaEngine:
         self.step_kernels = step_kernels
         dev = block_table.device
         self.layout = StagingLayout(self.L, self.B, self.hq, self.hkv, self.hidden)
-        self.staging = torch.zeros(self.layout.nbytes, dtype=torch.uint8, device=dev)
-        self.v = self.layout.views(self.staging)
+        # One staging buffer, or two: the even steps' graph reads slot 0, the odd steps' slot
+        # 1, so that step i + 1's inputs can be copied in while step i runs.
+        if staging_slots not in (1, 2):
+            raise ValueError("staging_slots must be 1 or 2")
+        self.slots = staging_slots
+        self.staging_bufs = [torch.zeros(self.layout.nbytes, dtype=torch.uint8, device=dev)
+                             for _ in range(staging_slots)]
+        self.staging = self.staging_bufs[0]
+        self.vs = [self.layout.views(b) for b in self.staging_bufs]
+        self.v = self.vs[0]
         self.seq_lens = self.v["seq_lens"]
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.stats = torch.zeros(oda.ODA_STATS_LEN, dtype=torch.int64, device=dev) if with_stats else None
-        self.kvs = [oda.make_kv(k, v, block_table, self.seq_lens, self.status, self.stats)
-                    for k, v in zip(self.k_caches, self.v_caches)]
+        self.kvs_by_slot = [[oda.make_kv(k, v, block_table, vs["seq_lens"], self.status, self.stats)
+                             for k, v in zip(self.k_caches, self.v_caches)] for vs in self.vs]
+        self.kvs = self.kvs_by_slot[0]
         self.out = [torch.zeros(self.B, self.hq, 128, dtype=torch.float32, device=dev)
                     for _ in range(self.L - 1)]
         self.h = [torch.zeros(self.B, self.hidden, dtype=torch.float32, device=dev) for _ in range(2)]
@@ -134,12 +143,12 @@ class OdaEngine:
         """An even/odd pair of step graphs over this engine's buffers with the given threshold
         and phase mask, owned by the caller (launch graphs[step % 2]; close both when done).
         The engine's own graphs are untouched."""
-        v = self.v
-        names = lambda p: [v["%s_%d" % (p, l)] for l in range(self.L)]
         graphs = []
         for parity in (0, 1):
+            v = self.vs[parity % self.slots]
+            names = lambda p: [v["%s_%d" % (p, l)] for l in range(self.L)]
             graphs.append(oda.StepGraph(
-                self.kvs, self.hq, self.sink, self.window, self.scale,
+                self.kvs_by_slot[parity % self.slots], self.hq, self.sink, self.window, self.scale,
                 names("q_local"), names("k_local"), names("v_local"),
                 names("q_full"), names("k_full"), names("v_full"),
                 self._layer_out(parity), self.h[parity], v["emb"], self.w1, self.b1, self.w2,
@@ -151,6 +160,14 @@ class OdaEngine:
                 use_conditional=self.use_conditional, timing_events=self.timing,
                 phases=phases, step_kernels=self.step_kernels))
         return graphs
+
+    def views_for(self, step: int) -> dict:
+        """Staging views that step `step`'s graph reads (fill them, or copy a whole staging
+        image into staging_for(step), before launching it)."""
+        return self.vs[step % self.slots]
+
+    def staging_for(self, step: int) -> torch.Tensor:
+        return self.staging_bufs[step % self.slots]
 
     def set_h_prev(self, h0: torch.Tensor, step: int = 0):
         """h_{t-1} that step `step` will read."""

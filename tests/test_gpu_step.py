@@ -31,14 +31,15 @@ def _logical(bits, bt, caps, hkv, d):
 
 
 def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02, timing=False,
-               step_kernels=oda.ODA_STEP_FULL_PERSISTENT, expect_kernels=None, **layer_ranges):
+               step_kernels=oda.ODA_STEP_FULL_PERSISTENT, expect_kernels=None, staging_slots=1,
+               **layer_ranges):
     lay = oda_synth.make_layout(w, extra_tokens=steps + 2, device="cuda", lengths=lengths)
     caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
     rw = oda_synth.make_recall_weights(w, device="cuda", std=recall_std)
     eng = OdaEngine([c[0] for c in caches], [c[1] for c in caches], lay.block_table,
                     w.num_q_heads, (rw.w1, rw.b1, rw.w2, rw.b2), theta, sink=w.sink,
                     window=w.window, use_conditional=use_conditional, timing=timing,
-                    step_kernels=step_kernels, **layer_ranges)
+                    step_kernels=step_kernels, staging_slots=staging_slots, **layer_ranges)
     if expect_kernels is not None:                  # launches per step: Local, gate, Full
         assert eng.graphs[0].kernels() == expect_kernels, eng.graphs[0].kernels()
     h0 = oda_synth.make_h0(w, device="cuda")
@@ -58,7 +59,7 @@ def _run_steps(w, lengths, steps, theta, use_conditional=True, recall_std=0.02, 
     n_phases = 0
     for i in range(steps):
         si = oda_synth.make_step_inputs(w, i, device="cuda")
-        fill_staging(eng.v, si, [n + i + 1 for n in lengths])
+        fill_staging(eng.views_for(i), si, [n + i + 1 for n in lengths])
         if timing:
             eng.set_events(i, evs)
         eng.launch(i)
@@ -330,3 +331,14 @@ def test_persistent_local_every_shape_matches_oracle(shape, hq, hkv, batch, leng
                    expect_kernels=expect)
     finally:
         oda.oda_debug_set_local_shape(-1)
+
+
+@pytest.mark.parametrize("step_kernels", [oda.ODA_STEP_FULL_PERSISTENT, oda.ODA_STEP_PERSISTENT])
+def test_two_staging_slots_match_oracle(step_kernels):
+    """Even and odd steps read their own staging slot (so that a step's inputs can be copied
+    in while the previous step runs); the decode is the oracle's either way."""
+    w = oda_synth.Workload(name="slots", layers=3, batch=2, num_q_heads=16, num_kv_heads=8,
+                           prefill=900, steps=5, seed=310, sink=4, window=128)
+    n = _run_steps(w, [900, 333], 5, theta=0.0, use_conditional=False, staging_slots=2,
+                   step_kernels=step_kernels)
+    assert 0 < n < 10
