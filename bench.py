@@ -1050,38 +1050,11 @@ def run_oda(args, dist: Dist):
         torch.cuda.synchronize()
         dist.barrier()
         fc_e = eng.full_count.clone()
-        # Two staging slots: step i's inputs go in on an input stream while step i - 1 runs,
-        # once the graph of step i - 2 (same slot) has finished; step i's selected output (its
-        # result) comes back on an output stream while step i + 1 runs, before step i + 2
-        # overwrites it. (One stream for both would queue step i + 1's inputs behind step i's
-        # output read, which waits for step i to finish.)
-        cs_in, cs_out = torch.cuda.Stream(), torch.cuda.Stream()
-        ran = [torch.cuda.Event() for _ in range(2)]      # step graph of this slot finished
-        staged = [torch.cuda.Event() for _ in range(2)]   # inputs of this slot copied in
-        read = [torch.cuda.Event() for _ in range(2)]     # outputs of this slot copied out
+        # through the engine's host path: inputs copied in and each step's result read out on
+        # their own streams, overlapping the steps (OdaEngine.run_from_host)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        cs_in.wait_stream(stream)
-        cs_out.wait_stream(stream)
-        for i in range(E2E):
-            k = step % 2
-            if i >= 2:
-                cs_in.wait_event(ran[k])
-            with torch.cuda.stream(cs_in):
-                eng.staging_for(step).copy_(host_pool[i], non_blocking=True)
-            staged[k].record(cs_in)
-            stream.wait_event(staged[k])
-            if i >= 2:
-                stream.wait_event(read[k])
-            eng.launch(step, stream)
-            ran[k].record(stream)
-            cs_out.wait_event(ran[k])
-            with torch.cuda.stream(cs_out):
-                out_h[i % 2].copy_(eng.selected_last(step), non_blocking=True)
-            read[k].record(cs_out)
-            step += 1
-        stream.wait_stream(cs_in)
-        stream.wait_stream(cs_out)
+        step = eng.run_from_host(host_pool, out_h, step, stream)
         b.record(stream)
         torch.cuda.synchronize()
         dist.barrier()

@@ -169,6 +169,45 @@ class OdaEngine:
     def staging_for(self, step: int) -> torch.Tensor:
         return self.staging_bufs[step % self.slots]
 
+    def run_from_host(self, host_inputs: torch.Tensor, out_host: torch.Tensor, first_step: int,
+                      stream=None) -> int:
+        """Decode len(host_inputs) steps from pinned host memory: step i's staging image
+        (host_inputs[i], uint8 [staging bytes]) goes in on an input stream while step i - 1
+        runs (needs two staging slots), and its selected last-layer output (its result, fp32
+        [B][hidden]) comes back into out_host[i % len(out_host)] on an output stream while step
+        i + 1 runs. Every copy and launch is queued without a host wait; returns the step
+        index after the last one. The caller synchronises before reading out_host."""
+        if self.slots != 2:
+            raise ValueError("run_from_host needs an engine with staging_slots=2")
+        stream = stream or torch.cuda.current_stream()
+        cs_in, cs_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ran = [torch.cuda.Event() for _ in range(2)]      # the graph of this slot finished
+        staged = [torch.cuda.Event() for _ in range(2)]   # this slot's inputs copied in
+        read = [torch.cuda.Event() for _ in range(2)]     # this slot's output copied out
+        cs_in.wait_stream(stream)
+        cs_out.wait_stream(stream)
+        step = first_step
+        for i in range(host_inputs.shape[0]):
+            k = step % 2
+            if i >= 2:
+                cs_in.wait_event(ran[k])          # step - 2 has read this slot
+            with torch.cuda.stream(cs_in):
+                self.staging_for(step).copy_(host_inputs[i], non_blocking=True)
+            staged[k].record(cs_in)
+            stream.wait_event(staged[k])
+            if i >= 2:
+                stream.wait_event(read[k])        # step - 2's output has been read out
+            self.launch(step, stream)
+            ran[k].record(stream)
+            cs_out.wait_event(ran[k])
+            with torch.cuda.stream(cs_out):
+                out_host[i % out_host.shape[0]].copy_(self.selected_last(step), non_blocking=True)
+            read[k].record(cs_out)
+            step += 1
+        stream.wait_stream(cs_in)
+        stream.wait_stream(cs_out)
+        return step
+
     def set_h_prev(self, h0: torch.Tensor, step: int = 0):
         """h_{t-1} that step `step` will read."""
         self.h[step % 2].copy_(h0)

@@ -342,3 +342,57 @@ def test_two_staging_slots_match_oracle(step_kernels):
     n = _run_steps(w, [900, 333], 5, theta=0.0, use_conditional=False, staging_slots=2,
                    step_kernels=step_kernels)
     assert 0 < n < 10
+
+
+def test_run_from_host_overlapped_matches_oracle():
+    """The host path users call (OdaEngine.run_from_host): each step's staging image comes
+    from pinned host memory on an input stream and its selected output goes back on an output
+    stream while the neighbouring steps run; every step's result, read back on the host, is
+    the oracle's. Recall weights large enough that no score sits within 1e-2 of theta (the
+    gates are not read back)."""
+    from sparse_kv_recall_b200.engine import StagingLayout
+    w = oda_synth.Workload(name="host-path", layers=3, batch=2, num_q_heads=16, num_kv_heads=8,
+                           prefill=700, steps=6, seed=320, sink=4, window=128)
+    lengths = [700, 250]
+    lay = oda_synth.make_layout(w, extra_tokens=w.steps + 2, device="cuda", lengths=lengths)
+    caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
+    rw = oda_synth.make_recall_weights(w, device="cuda", std=0.5)
+    eng = OdaEngine([c[0] for c in caches], [c[1] for c in caches], lay.block_table,
+                    w.num_q_heads, (rw.w1, rw.b1, rw.w2, rw.b2), 0.0, sink=w.sink,
+                    window=w.window, use_conditional=False, staging_slots=2)
+    h0 = oda_synth.make_h0(w, device="cuda")
+    eng.set_h_prev(h0, 0)
+    bt = lay.block_table.cpu().numpy()
+    dec = O.OdaDecoder([_logical(oda_synth.bf16_bits(k), bt, lay.capacity, w.num_kv_heads, 128)
+                        for k, _ in caches],
+                       [_logical(oda_synth.bf16_bits(v), bt, lay.capacity, w.num_kv_heads, 128)
+                        for _, v in caches],
+                       lengths, h0.double().cpu().numpy(),
+                       (rw.w1.double().cpu().numpy(), rw.b1.double().cpu().numpy(),
+                        rw.w2.double().cpu().numpy(), rw.b2), sink=w.sink, window=w.window,
+                       theta=0.0)
+    layout = StagingLayout(w.layers, w.batch, w.num_q_heads, w.num_kv_heads, w.hidden)
+    host = torch.empty((w.steps, layout.nbytes), dtype=torch.uint8, pin_memory=True)
+    scratch = torch.zeros(layout.nbytes, dtype=torch.uint8, device="cuda")
+    inputs = []
+    for i in range(w.steps):
+        si = oda_synth.make_step_inputs(w, i, device="cuda")
+        fill_staging(layout.views(scratch), si, [n + i + 1 for n in lengths])
+        host[i].copy_(scratch)
+        inputs.append(si)
+    out_host = torch.empty((w.steps, w.batch, w.hidden), dtype=torch.float32, pin_memory=True)
+    assert eng.run_from_host(host, out_host, 0) == w.steps
+    torch.cuda.synchronize()
+    assert int(eng.status.item()) == 0
+    n_gated = 0
+    for i, si in enumerate(inputs):
+        inp = {k: [oda_synth.bf16_bits(x) for x in getattr(si, k)]
+               for k in ("q_local", "k_local", "v_local", "q_full", "k_full", "v_full")}
+        inp["emb"] = si.emb.double().cpu().numpy()
+        ref, _, rq, rg = dec.step(inp)
+        assert np.abs(rq).min() >= 1e-2, rq                   # no near-tie: the gate is sure
+        assert_attn_close(out_host[i].numpy().reshape(w.batch, w.num_q_heads, 128)[None],
+                          ref[-1][None], "host path step %d" % i)
+        n_gated += int(rg.sum())
+    assert eng.full_count.cpu().tolist()[0] == n_gated
+    eng.close()
