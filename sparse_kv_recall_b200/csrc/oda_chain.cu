@@ -131,14 +131,6 @@ __device__ __forceinline__ float ld_keep(const float* p, uint64_t pol) {
   return v;
 }
 
-// Cluster barrier halves (all threads of every CTA of the cluster).
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 // Thread 0 waits for the launch-wide count to reach `target`; on a timeout it reports
 // ODA_DEV_TIMEOUT and raises the abort word. Returns the answer to every thread of the CTA.
 __device__ __forceinline__ bool cta_wait_count(unsigned* ctr, unsigned target,
@@ -476,7 +468,7 @@ __global__ void __launch_bounds__(W * 32, (C == 16 && G != 4) ? 2 : 1)
 #pragma unroll
         for (int c2 = 0; c2 < C; ++c2) M = fmaxf(M, inbox[c2 * stride + kOut + gg]);
         const float lc = inbox[cc * stride + kOut + gg];
-        wsm[tid] = (lc == -INFINITY) ? 0.f : exp2f(lc - M);
+        wsm[tid] = (lc == -INFINITY) ? 0.f : ex2_fast(lc - M);
         if (cc == 0) msm[gg] = M;
       }
       __syncthreads();
@@ -497,10 +489,10 @@ __global__ void __launch_bounds__(W * 32, (C == 16 && G != 4) ? 2 : 1)
             ov[2] = fmaf(wc, av.z, ov[2]);
             ov[3] = fmaf(wc, av.w, ov[3]);
           }
-          const float rL = 1.f / Ls;
+          const float rL = rcp_fast(Ls);
 #pragma unroll
           for (int k = 0; k < 4; ++k) ov[k] *= rL;
-          l2 = M + log2f(Ls);
+          l2 = M + lg2_fast(Ls);
         }
         const size_t h = (size_t)b * p.hq + g * G + gg;
         float* dst = ly.out + h * kHeadDim + d;

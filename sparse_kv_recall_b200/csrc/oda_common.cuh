@@ -32,6 +32,28 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
 }
 
+// ---- softmax arithmetic -------------------------------------------------------------------
+// Base-2 exponential, reciprocal and base-2 logarithm by the PTX approximate instructions
+// (ex2.approx, rcp.approx, lg2.approx; flush to zero): a few ulp from the exact values, where
+// the library calls take several times as many instructions. Softmax weights and rescale
+// factors (arguments <= 0, results in [0, 1]), and the merges' 1 / L and log2 L for L >= 1,
+// sit on the decode kernels' latency-bound chains.
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_fast(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_fast(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---- shared-memory barriers and 1-D bulk copies (TMA engine, no tensor map, no multicast) -
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -134,6 +156,32 @@ __device__ __forceinline__ unsigned cluster_ctarank() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
+}
+// The halves of a cluster barrier (all threads of every CTA of the cluster): arrive with
+// release, arrive without ordering (after fence_barrier_init it publishes mbarrier
+// initialisation), and wait with acquire.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 16-byte and 4-byte stores into the shared memory of a CTA of the cluster (`dst` from
+// cluster_addr), each completing its bytes on that CTA's mbarrier `bar` (also from
+// cluster_addr): the receiver learns from the barrier phase that every expected byte landed.
+__device__ __forceinline__ void st_async4(uint32_t dst, float4 v, uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async1(uint32_t dst, float v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];"
+               ::"r"(dst), "f"(v), "r"(bar)
+               : "memory");
 }
 __device__ __forceinline__ void dsmem_st(float* local, unsigned rank, float v) {
   uint32_t remote;

@@ -36,27 +36,43 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
 // Short-window kernel (Local at small batch). The split above ends a short launch with a
 // chain of global round trips: every CTA's partial to global memory, an acquire-release
 // ticket, the last CTA reading every partial back. Here one thread-block cluster of
-// kClusterCtas CTAs takes one (sequence, KV head); each of its kClusterCtas x kClusterWarps
-// warps attends at most one page, and the CTAs' partials are merged through distributed
-// shared memory by cluster rank 0 after one cluster barrier. The page step, the commit of
-// slot t and the in-CTA merge are those of the split pass.
+// kLocalCtas CTAs takes one (sequence, KV head). Ranks 1 .. kLocalCtas - 1 hold the pages,
+// one per warp (kLocalClusterPages at most); each forms its CTA partial and sends it straight
+// into rank 0's shared memory by st.async stores that complete on rank 0's inbox mbarrier, and
+// leaves. Rank 0 holds no page: its stage memory is that inbox; once the barrier phase shows
+// every partial landed it merges them in rank order and writes the output. No CTA waits for
+// another except rank 0 for the partials (the cluster barrier is only split around the
+// launch, to publish the mbarrier's initialisation before the first remote store), so a
+// CTA's SM slot frees as soon as its partial is sent, for the next layer's clusters. The page
+// step (tensor-core scores for G = 2 and 4), the commit of slot t and the in-CTA merge are
+// those of the split pass and the persistent Local kernel.
 // ---------------------------------------------------------------------------------------
 template <int G>
-__global__ void __launch_bounds__(kClusterThreads, 2) cluster_decode_kernel(const DecodeParams p) {
-  constexpr int VPL = Vpl<G>::value;
+__global__ void __launch_bounds__(kLocalThreads, kLocalCtasPerSm)
+    cluster_decode_kernel(const DecodeParams p) {
+  constexpr bool kMma = MmaScores<G>::value;
+  constexpr int VPL = ClusterStates<G, kMma>::VPL;
   constexpr int kPs = 18 * G;
+  constexpr int kPart = ClusterPart<G>::value;
+  static_assert(kLocalCtas * kPart * sizeof(float) <= kLocalWarps * kStageBytes,
+                "rank 0's inbox lives in its stage memory");
+  static_assert(cluster_scratch_floats<G, kMma, kLocalWarps>() * sizeof(float) <=
+                    kLocalWarps * kStageBytes,
+                "the in-CTA merge reuses the stage memory");
   extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* stages = smem;  // [warp][kStageBytes]: one page per warp
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kClusterWarps * kStageBytes);
-  float* pscratch = reinterpret_cast<float*>(bars + kClusterWarps);  // [warp][kPs]
-  // rank 0's copy gathers every CTA's partial: [kClusterCtas][G * 128 outputs + G log-sums]
-  float* part = align16(pscratch + kClusterWarps * kPs);
+  unsigned char* stages = smem;  // [warp][kStageBytes]: one page per warp (ranks >= 1)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kLocalWarps * kStageBytes);
+  float* pscratch = reinterpret_cast<float*>(bars + kLocalWarps);  // [warp][kPs]
+  // rank 0: [kLocalCtas][kPart] partials (slot r from rank r; slot 0 unused)
+  float* inbox = reinterpret_cast<float*>(stages);
   __shared__ unsigned long long s_rows, s_pages;
+  __shared__ __align__(8) uint64_t s_inbar;  // rank 0: every partial has landed
+  constexpr uint32_t kPartBytes = (ClusterPart<G>::kOut + G) * sizeof(float);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int li = lane & 15;
   const unsigned rank = cluster_ctarank();
-  const int bg = blockIdx.x / kClusterCtas;
+  const int bg = blockIdx.x / kLocalCtas;
   const int b = bg / p.hkv, g = bg % p.hkv;
   if (tid == 0) {
     s_rows = 0;
@@ -64,16 +80,21 @@ __global__ void __launch_bounds__(kClusterThreads, 2) cluster_decode_kernel(cons
   }
   if (lane == 0) {
     mbar_init(&bars[warp], 1);
+    if (tid == 0 && rank == 0) {
+      mbar_init(&s_inbar, 1);
+      mbar_arrive_expect_tx(&s_inbar, (kLocalCtas - 1) * kPartBytes);
+    }
     fence_barrier_init();
   }
   __syncwarp();
+  cluster_arrive_relaxed();  // rank 0's inbox barrier is initialised (waited for before a push)
   if (p.wait_first) griddep_wait();
 
   // Before the dependency wait: the plan and this warp's page copy (history pages only).
   const SeqPlan sp = make_plan(p.plan, b);
   if (rank == 0 && g == 0 && tid == 0 && sp.err != 0) report(p.status, sp.err);
-  const int j = (int)rank * kClusterWarps + warp;
-  const bool has = !sp.skip && j < sp.npages;
+  const int j = ((int)rank - 1) * kLocalWarps + warp;
+  const bool has = rank != 0 && !sp.skip && j < sp.npages;
   const size_t head_off = (size_t)g * (kPage * kHeadDim);
   const size_t page_stride = (size_t)p.hkv * kPage * kHeadDim;
   unsigned char* st = stages + warp * kStageBytes;
@@ -113,19 +134,26 @@ __global__ void __launch_bounds__(kClusterThreads, 2) cluster_decode_kernel(cons
   unsigned rows_vis = 0, pages_read = 0;
   if (has && r.err == 0) {
     f2_t q2[G][4];
-    load_q_scaled<G>(p.q, p.hq, b, g, p.scale_log2, li, q2);
+    uint4 qv[4];
+    if constexpr (kMma) load_q_mma<G>(p.q + ((size_t)b * p.hq + g * G) * kHeadDim, lane, qv);
+    else load_q_scaled<G>(p.q, p.hq, b, g, p.scale_log2, li, q2);
     if (!__all_sync(0xffffffffu, mbar_wait(&bars[warp], 0u, p.wait_ns))) {
       if (lane == 0) report(p.status, ODA_DEV_TIMEOUT);
     } else {
       if (p.k_new != nullptr && r.lp == sp.t / kPage)
         commit_slot(st, p.k_new, p.v_new, p.k_cache_w, p.v_cache_w, b, p.hkv, g, sp.t, r.pb,
                     lane);
-      page_step<G>(st, q2, m_run, l_run, acc, pscratch + warp * kPs, sp, r.lp, lane, rows_vis);
+      if constexpr (kMma)
+        page_step_mma<G>(st, qv, p.scale_log2, m_run, l_run, acc, pscratch + warp * kPs, sp,
+                         r.lp, lane, rows_vis);
+      else
+        page_step<G>(st, q2, m_run, l_run, acc, pscratch + warp * kPs, sp, r.lp, lane,
+                     rows_vis);
       pages_read = 1;
     }
   }
 
-  // ---- merge the CTA's 2 x kClusterWarps half-warp states, push to rank 0 ----
+  // ---- merge the CTA's warp states, push to rank 0 ----
   if (p.stats != nullptr && lane == 0 && pages_read) {
     atomicAdd(&s_rows, (unsigned long long)rows_vis);
     atomicAdd(&s_pages, (unsigned long long)pages_read);
@@ -135,13 +163,19 @@ __global__ void __launch_bounds__(kClusterThreads, 2) cluster_decode_kernel(cons
     if (s_rows) atomicAdd(&p.stats[ODA_STAT_ROWS], s_rows);
     if (s_pages) atomicAdd(&p.stats[ODA_STAT_PAGES], s_pages);
   }
-  cluster_push_partial<G>(m_run, l_run, acc, reinterpret_cast<float*>(stages), part,
-                          ClusterPart<G>::value, rank);
-  cluster_sync();  // every CTA's partial has landed in rank 0's shared memory
-  if (rank == 0 && !sp.skip && tid < kHeadDim) {
-    float o[G], l2[G];
-    cluster_merge_inbox<G>(part, ClusterPart<G>::value, o, l2);
-    write_final<G>(p, b, g, o, l2);
+  cluster_wait();  // (long since complete: every CTA arrived at its start)
+  if (rank != 0) {
+    cluster_push_partial<G, kMma, kLocalWarps, false, true>(
+        m_run, l_run, acc, reinterpret_cast<float*>(stages), inbox, kPart, rank,
+        cluster_addr(&s_inbar, 0));
+  } else if (tid < kHeadDim) {
+    if (!mbar_wait_cluster(&s_inbar, 0u, p.wait_ns)) {
+      if (tid == 0) report(p.status, ODA_DEV_TIMEOUT);
+    } else if (!sp.skip) {
+      float o[G], l2[G];
+      cluster_merge_inbox<G, 1, kLocalCtas>(inbox, kPart, o, l2);
+      write_final<G>(p, b, g, o, l2);
+    }
   }
 }
 
@@ -171,6 +205,10 @@ __global__ void visible_mask_kernel(PlanArgs a, uint8_t* mask, int max_tokens, i
 // ---------------------------------------------------------------------------------------
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// The CTAs of a Local cluster on distinct SMs where the hardware can: their page steps are
+// bound by instruction issue, so two of one cluster on one SM take turns.
+constexpr cudaClusterSchedulingPolicy kLocalClusterPolicy = cudaClusterSchedulingPolicySpread;
+
 static size_t decode_smem_bytes(int G) { return split_smem_bytes(G); }
 
 // Decode workspace: split partials (O and log-sums, one slot per CTA and per (b, g)), the
@@ -190,11 +228,13 @@ static WsLayout ws_layout(int batch, int hkv, int G, int grid) {
   return w;
 }
 
+// Stages (rank 0: the inbox), one mbarrier and the softmax exchange per warp (73.3 KB at
+// G = 2, 74.6 KB at G = 4), padded to kLocalSmemFloor: two CTAs per SM.
 static size_t cluster_smem_bytes(int G) {
-  const int part = (G * kHeadDim + G + 3) / 4 * 4;  // ClusterPart<G>::value
-  return (size_t)kClusterWarps * kStageBytes + (size_t)kClusterWarps * sizeof(uint64_t) +
-         (size_t)kClusterWarps * 18 * G * sizeof(float) + 16 +
-         (size_t)kClusterCtas * part * sizeof(float);
+  const size_t need = (size_t)kLocalWarps * kStageBytes +
+                      (size_t)kLocalWarps * sizeof(uint64_t) +
+                      (size_t)kLocalWarps * 18 * G * sizeof(float);
+  return need > kLocalSmemFloor ? need : kLocalSmemFloor;
 }
 
 // Clusters of the short-window kernel the device can hold at once, per device and group
@@ -216,16 +256,18 @@ static int prepare_decode_kernel(int device) {
                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess)
     return cuda_status(e);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kClusterCtas);
-  cfg.blockDim = dim3(kClusterThreads);
+  cfg.gridDim = dim3(kLocalCtas);
+  cfg.blockDim = dim3(kLocalThreads);
   cfg.dynamicSmemBytes = cluster_smem_bytes(G);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kClusterCtas;
+  attr[0].val.clusterDim.x = kLocalCtas;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+  attr[1].val.clusterSchedulingPolicyPreference = kLocalClusterPolicy;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, cluster_decode_kernel<G>, &cfg) != cudaSuccess) {
     cudaGetLastError();  // not fatal: the split kernel serves every launch
@@ -312,18 +354,20 @@ static cudaError_t launch_cluster_kernel(const DecodeParams& p, int grid, cudaSt
                                          bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kClusterThreads);
+  cfg.blockDim = dim3(kLocalThreads);
   cfg.dynamicSmemBytes = cluster_smem_bytes(G);
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kClusterCtas;
+  attr[0].val.clusterDim.x = kLocalCtas;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+  attr[1].val.clusterSchedulingPolicyPreference = kLocalClusterPolicy;
+  attr[2].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[2].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 2 : 1;
+  cfg.numAttrs = pdl ? 3 : 2;
   return cudaLaunchKernelEx(&cfg, cluster_decode_kernel<G>, p);
 }
 
@@ -335,7 +379,7 @@ static bool use_cluster_kernel(const oda_kv* kv, const oda_visibility& vis, cons
   if (vis.mode != ODA_MODE_LOCAL) return false;
   const long long pages = (vis.sink + kPage - 1) / kPage + (long long)(vis.window - 1) / kPage + 2;
   const long long clusters = (long long)kv->batch * kv->num_kv_heads;
-  return pages <= kClusterPages && clusters * kClusterCtas <= 2ll * di.sms &&
+  return pages <= kLocalClusterPages && clusters * kLocalCtas <= 2ll * di.sms &&
          clusters <= g_max_clusters[di.device][G];
 }
 
@@ -476,7 +520,7 @@ int launch_decode(const oda_kv* kv, const oda_visibility& vis, const void* q, in
   }
   if (rc != ODA_OK) return rc;
   const bool cluster = use_cluster_kernel(kv, vis, di, G);
-  const int cgrid = kv->batch * kv->num_kv_heads * kClusterCtas;
+  const int cgrid = kv->batch * kv->num_kv_heads * kLocalCtas;
   cudaError_t e;
   switch (G) {
     case 1:

@@ -150,8 +150,8 @@ __device__ __forceinline__ void page_step(const unsigned char* stage, const f2_t
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     const float mnew = fmaxf(m_run[u], mx);
-    const float pr = (v == -INFINITY) ? 0.f : exp2f(v - mnew);
-    const float al = (m_run[u] == mnew) ? 1.f : exp2f(m_run[u] - mnew);
+    const float pr = (v == -INFINITY) ? 0.f : ex2_fast(v - mnew);
+    const float al = (m_run[u] == mnew) ? 1.f : ex2_fast(m_run[u] - mnew);
     l_run[u] = l_run[u] * al + pr;
     m_run[u] = mnew;
     const int gh = (G >= 2) ? ((li & 1) * (G / 2) + u) : 0;
@@ -275,7 +275,7 @@ __device__ __forceinline__ void page_step_mma(const unsigned char* stage, const 
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       const bool up = mx > m_run[u] + kLazyMax;
-      const float al = !up ? 1.f : (m_run[u] == -INFINITY ? 0.f : exp2f(m_run[u] - mx));
+      const float al = !up ? 1.f : (m_run[u] == -INFINITY ? 0.f : ex2_fast(m_run[u] - mx));
       if (up) m_run[u] = mx;
       l_run[u] *= al;
       if (head_ok && gid == 0) ashare[2 * tig + u] = al;
@@ -287,7 +287,7 @@ __device__ __forceinline__ void page_step_mma(const unsigned char* stage, const 
     const int slot = (r & 1) * 8 + (r >> 1);  // page_step's [half][k] order of row r
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const float pr = (s[t][u] == -INFINITY) ? 0.f : exp2f(s[t][u] - m_run[u]);
+      const float pr = (s[t][u] == -INFINITY) ? 0.f : ex2_fast(s[t][u] - m_run[u]);
       l_run[u] += pr;
       if (head_ok) pshare[slot * G + 2 * tig + u] = pr;
     }
@@ -695,12 +695,12 @@ __device__ __forceinline__ void decode_pass(const DecodeParams& p, const SplitSm
 #pragma unroll
         for (int s = 0; s < 2 * kWarps; ++s) {
           const float ms = Mw[s * G + gg];
-          const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+          const float w = (ms == -INFINITY) ? 0.f : ex2_fast(ms - M);
           L = fmaf(w, Lw[s * G + gg], L);
           a = fmaf(w, Aw[(s * G + gg) * kHeadDim + tid], a);
         }
-        o[gg] = a / L;
-        l2[gg] = M + log2f(L);
+        o[gg] = a * rcp_fast(L);
+        l2[gg] = M + lg2_fast(L);
       }
     }
 
@@ -751,7 +751,7 @@ __device__ __forceinline__ void decode_pass(const DecodeParams& p, const SplitSm
           float sum = 0.f;
           for (int s = lane; s < n_contrib; s += 32) {
             const float ls = sw[s * G + warp];
-            const float wgt = (ls == -INFINITY) ? 0.f : exp2f(ls - m);
+            const float wgt = (ls == -INFINITY) ? 0.f : ex2_fast(ls - m);
             sw[s * G + warp] = wgt;
             sum += wgt;
           }
@@ -786,8 +786,8 @@ __device__ __forceinline__ void decode_pass(const DecodeParams& p, const SplitSm
             o[gg] = 0.f;
             l2[gg] = -INFINITY;
           } else {
-            o[gg] = a[gg] / L;
-            l2[gg] = M + log2f(L);
+            o[gg] = a[gg] * rcp_fast(L);
+            l2[gg] = M + lg2_fast(L);
           }
         }
         write_final<G>(p, b, g, o, l2);
@@ -833,6 +833,16 @@ constexpr int kClusterCtas = 16;  // a non-portable cluster size (B200 supports 
 constexpr int kClusterWarps = 9;
 constexpr int kClusterThreads = kClusterWarps * 32;
 constexpr int kClusterPages = kClusterCtas * kClusterWarps;  // pages per (b, g) at most
+// The per-layer cluster kernel: rank 0 holds no page (its stage memory is the inbox); two CTAs
+// per SM (its shared memory is padded to kLocalSmemFloor so that a third does not fit: with
+// three, every cluster of the next layer is resident early, but the layer itself was measured
+// slower, 5.50 against 5.28 us at 28 layers x 8 KV heads x 2,052 tokens).
+constexpr int kLocalCtas = 16;
+constexpr int kLocalWarps = 9;
+constexpr int kLocalThreads = kLocalWarps * 32;
+constexpr int kLocalClusterPages = (kLocalCtas - 1) * kLocalWarps;
+constexpr int kLocalCtasPerSm = 2;
+constexpr size_t kLocalSmemFloor = 80 * 1024;  // > 228 KB per SM / 3 - 1 KB reserved per CTA
 
 // Floats of one CTA partial in rank 0's inbox: G * 128 outputs + G log-sums, padded to a
 // multiple of 4 so that every slot starts 16-byte aligned (the partials arrive by 16-byte
@@ -896,7 +906,7 @@ struct ClusterStates {
 
 // Floats of the in-CTA merge scratch for ClusterStates<G, kMma, W>::value states.
 template <int G, bool kMma, int W = kClusterWarps>
-constexpr int cluster_scratch_floats() {
+__host__ __device__ constexpr int cluster_scratch_floats() {
   return ClusterStates<G, kMma, W>::value * G * (kHeadDim + 2);
 }
 
@@ -905,13 +915,16 @@ constexpr int cluster_scratch_floats() {
 // from earlier reads of it), normalises, and stores the result and its log2-sum into slot
 // `rank` (slots `stride` floats apart) of cluster rank 0's inbox (`inbox` is the local
 // address of the inbox; every CTA of the cluster has one at the same offset), the caller's
-// cluster barrier publishing the stores -- or, with kLocal, into this CTA's own buffer
-// `inbox` for the caller to ship. Contains a CTA barrier before the states are read.
-template <int G, bool kMma = false, int W = kClusterWarps, bool kLocal = false>
+// cluster barrier publishing the stores -- or, with kAsync, by st.async stores that complete
+// on rank 0's mbarrier `inbar` (a cluster address), (G * 128 + G) * 4 bytes per CTA -- or, with
+// kLocal, into this CTA's own buffer `inbox` for the caller to ship. Contains a CTA barrier
+// before the states are read.
+template <int G, bool kMma = false, int W = kClusterWarps, bool kLocal = false,
+          bool kAsync = false>
 __device__ __forceinline__ void cluster_push_partial(
     const float (&m_run)[ClusterStates<G, kMma, W>::VPL],
     const float (&l_run)[ClusterStates<G, kMma, W>::VPL], f2_t (&acc)[G][4], float* scratch,
-    float* inbox, int stride, unsigned rank) {
+    float* inbox, int stride, unsigned rank, uint32_t inbar = 0u) {
   constexpr int VPL = ClusterStates<G, kMma, W>::VPL;
   constexpr int kStates = ClusterStates<G, kMma, W>::value;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1009,7 +1022,7 @@ __device__ __forceinline__ void cluster_push_partial(
 #pragma unroll
       for (int s2 = 0; s2 < kStates; ++s2) {
         const float ms = Mw[s2 * G + gg];
-        const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+        const float w = (ms == -INFINITY) ? 0.f : ex2_fast(ms - M);
         L = fmaf(w, Lw[s2 * G + gg], L);
         const float4 av = *reinterpret_cast<const float4*>(Aw + (s2 * G + gg) * kHeadDim + d);
         a.x = fmaf(w, av.x, a.x);
@@ -1017,13 +1030,16 @@ __device__ __forceinline__ void cluster_push_partial(
         a.z = fmaf(w, av.z, a.z);
         a.w = fmaf(w, av.w, a.w);
       }
-      const float rL = 1.f / L;
+      const float rL = rcp_fast(L);
       oval = make_float4(a.x * rL, a.y * rL, a.z * rL, a.w * rL);
-      l2 = M + log2f(L);
+      l2 = M + lg2_fast(L);
     }
     if constexpr (kLocal) {  // into this CTA's own slot (`inbox`), shipped by the caller
       *reinterpret_cast<float4*>(inbox + 4 * o4) = oval;
       if (d == 0) inbox[kOut + gg] = l2;
+    } else if constexpr (kAsync) {
+      st_async4(cluster_addr(slot + 4 * o4, 0), oval, inbar);
+      if (d == 0) st_async1(cluster_addr(slot + kOut + gg, 0), l2, inbar);
     } else {
       dsmem_st4(slot + 4 * o4, 0, oval);
       if (d == 0) dsmem_st(slot + kOut + gg, 0, l2);
@@ -1031,40 +1047,41 @@ __device__ __forceinline__ void cluster_push_partial(
   }
 }
 
-// Rank 0's merge of the kClusterCtas partials in its inbox (slots `stride` floats apart), in
-// rank order: dim `tid` (< 128) of every head of the group.
-template <int G>
+// Rank 0's merge of the partials in slots kFirst .. C - 1 of its inbox (slots `stride` floats
+// apart), in rank order: dim `tid` (< 128) of every head of the group.
+template <int G, int kFirst = 0, int C = kClusterCtas>
 __device__ __forceinline__ void cluster_merge_inbox(const float* inbox, int stride, float (&o)[G],
                                                     float (&l2)[G]) {
   constexpr int kOut = ClusterPart<G>::kOut;
+  constexpr int kN = C - kFirst;
   const int kPart = stride;
   const int tid = threadIdx.x;
-  float ls[G][kClusterCtas], os[G][kClusterCtas];
+  float ls[G][kN], os[G][kN];
 #pragma unroll
   for (int gg = 0; gg < G; ++gg)
 #pragma unroll
-    for (int c = 0; c < kClusterCtas; ++c) {
-      ls[gg][c] = inbox[c * kPart + kOut + gg];
-      os[gg][c] = inbox[c * kPart + gg * kHeadDim + tid];
+    for (int c = 0; c < kN; ++c) {
+      ls[gg][c] = inbox[(c + kFirst) * kPart + kOut + gg];
+      os[gg][c] = inbox[(c + kFirst) * kPart + gg * kHeadDim + tid];
     }
 #pragma unroll
   for (int gg = 0; gg < G; ++gg) {
     float M = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < kClusterCtas; ++c) M = fmaxf(M, ls[gg][c]);
+    for (int c = 0; c < kN; ++c) M = fmaxf(M, ls[gg][c]);
     if (M == -INFINITY) {
       o[gg] = 0.f;
       l2[gg] = -INFINITY;
     } else {
       float L = 0.f, a = 0.f;
 #pragma unroll
-      for (int c = 0; c < kClusterCtas; ++c) {
-        const float w = (ls[gg][c] == -INFINITY) ? 0.f : exp2f(ls[gg][c] - M);
+      for (int c = 0; c < kN; ++c) {
+        const float w = (ls[gg][c] == -INFINITY) ? 0.f : ex2_fast(ls[gg][c] - M);
         L += w;
         a = fmaf(w, os[gg][c], a);
       }
-      o[gg] = a / L;
-      l2[gg] = M + log2f(L);
+      o[gg] = a * rcp_fast(L);
+      l2[gg] = M + lg2_fast(L);
     }
   }
 }

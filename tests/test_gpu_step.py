@@ -265,9 +265,10 @@ def test_shapes_outside_the_persistent_local_kernel_fall_back():
 def test_persistent_step_equals_per_layer(theta, prefill):
     """The persistent Full kernel runs the per-layer split pass itself, so with every step
     recomputed by Full (theta = -inf) every layer output is bitwise the per-layer launches'.
-    The persistent Local kernel forms its page scores on the tensor cores and merges one state
-    per warp (the per-layer cluster kernel: CUDA-core scores, two states per warp), so Local
-    outputs (theta = +inf) agree to fp32 rounding. The default mode (Local per layer, Full
+    Both Local kernels form page scores on the tensor cores, but the persistent one spreads a
+    window's pages over all 16 CTAs of its cluster and the per-layer one over 15 (its rank 0
+    only merges), so the partials group differently and Local outputs (theta = +inf) agree to
+    fp32 rounding. The default mode (Local per layer, Full
     persistent) equals the per-layer launches bitwise at both ends. Committed K/V bits and the
     attended-row and page counters are identical either way; theta at +-inf keeps the gate out
     of it (the fused recall head sums in another order than the recall kernel). The 9000-token
