@@ -88,6 +88,9 @@ __global__ void __launch_bounds__(kLocalThreads, kLocalCtasPerSm)
   }
   __syncwarp();
   cluster_arrive_relaxed();  // rank 0's inbox barrier is initialised (waited for before a push)
+  // The next kernel (the next layer, or the recall head) may launch as soon as every CTA of
+  // this one is resident: its own pre-wait reads touch nothing this one writes.
+  griddep_launch_dependents();
   if (p.wait_first) griddep_wait();
 
   // Before the dependency wait: the plan and this warp's page copy (history pages only).
@@ -118,7 +121,6 @@ __global__ void __launch_bounds__(kLocalThreads, kLocalCtasPerSm)
   }
   __syncwarp();
   if (!p.wait_first) griddep_wait();
-  griddep_launch_dependents();
 
   float m_run[VPL], l_run[VPL];
   f2_t acc[G][4];
