@@ -390,11 +390,13 @@ void oda_step_graph_destroy(oda_step_graph* graph);
  * oda_debug_set_stall: ODA_STALL_DECODE_RING makes one stage of CTA 0's first warp in each
  * split decode launch wait for bytes that no copy delivers; ODA_STALL_LOCAL_CHAIN makes the
  * first cluster of the persistent Local kernel withhold its layer-0 count; ODA_STALL_FULL_CHAIN
- * makes CTA 0 of the persistent Full kernel withhold its layer-0 arrival. ODA_STALL_NONE (the
+ * makes CTA 0 of the persistent Full kernel withhold its layer-0 arrival; ODA_STALL_LOCAL_PUSH
+ * makes cluster rank 1 of the first cluster of the per-layer Local cluster kernel withhold its
+ * partial, so that rank 0's wait for its inbox runs out. ODA_STALL_NONE (the
  * default) turns the hook off. After a timeout the decode workspace must be zero-filled again.
  * Both return ODA_OK, or ODA_ERR_INVALID_ARG for an unknown kind. */
 enum { ODA_STALL_NONE = 0, ODA_STALL_DECODE_RING = 1, ODA_STALL_LOCAL_CHAIN = 2,
-       ODA_STALL_FULL_CHAIN = 3 };
+       ODA_STALL_FULL_CHAIN = 3, ODA_STALL_LOCAL_PUSH = 4 };
 int oda_debug_set_wait_limit(unsigned long long ns);
 int oda_debug_set_stall(int kind);
 /* Tuning hook: the shape of the persistent Local kernel in step graphs created after the call:

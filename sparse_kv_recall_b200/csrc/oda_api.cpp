@@ -33,7 +33,7 @@ extern "C" int oda_debug_set_local_shape(int index) {
 }
 
 extern "C" int oda_debug_set_stall(int kind) {
-  if (kind < ODA_STALL_NONE || kind > ODA_STALL_FULL_CHAIN) return ODA_ERR_INVALID_ARG;
+  if (kind < ODA_STALL_NONE || kind > ODA_STALL_LOCAL_PUSH) return ODA_ERR_INVALID_ARG;
   oda::g_stall.store(kind, std::memory_order_relaxed);
   return ODA_OK;
 }

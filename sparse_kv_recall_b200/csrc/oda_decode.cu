@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kLocalThreads, kLocalCtasPerSm)
     if (s_pages) atomicAdd(&p.stats[ODA_STAT_PAGES], s_pages);
   }
   cluster_wait();  // (long since complete: every CTA arrived at its start)
-  if (rank != 0) {
+  if (rank != 0 && !(p.test_stall == 2 && bg == 0 && rank == 1)) {
     cluster_push_partial<G, kMma, kLocalWarps, false, true>(
         m_run, l_run, acc, reinterpret_cast<float*>(stages), inbox, kPart, rank,
         cluster_addr(&s_inbar, 0));
@@ -496,7 +496,9 @@ int decode_params(const oda_kv* kv, const oda_visibility& vis, const void* q, in
   p.stats = kv->stats;
   p.wait_first = 0;
   p.wait_ns = test_wait_ns();
-  p.test_stall = test_stall() == ODA_STALL_DECODE_RING ? 1 : 0;
+  p.test_stall = test_stall() == ODA_STALL_DECODE_RING ? 1
+                 : test_stall() == ODA_STALL_LOCAL_PUSH ? 2
+                                                         : 0;
   return ODA_OK;
 }
 

@@ -48,7 +48,9 @@ struct DecodeParams {
   int wait_first;              // 1: the previous kernel may still write the gate: wait at once
   unsigned long long wait_ns;  // limit of every bounded wait (kWaitNs unless a test sets it)
   int test_stall;              // test hook: 1 = CTA 0's warp 0 arms its first stage for bytes
-                               // that no copy delivers, so that its bounded wait runs out
+                               // that no copy delivers, so that its bounded wait runs out;
+                               // 2 = the Local cluster kernel's first cluster's rank 1
+                               // withholds its partial, so that rank 0's inbox wait runs out
 };
 
 // ---- reduce-scatter of C values over the 16 lanes of a half-warp ------------------------
@@ -532,7 +534,7 @@ __device__ __forceinline__ void decode_pass(const DecodeParams& p, const SplitSm
       const PageRef r = page_ref(p.plan, sp, b, j);
       uint64_t* bar = &wbar[(wcount + n) % kStages];
       unsigned char* dst = wst + ((wcount + n) % kStages) * kStageBytes;
-      if (p.test_stall && c == 0 && warp == 0 && wcount + n == 0) {
+      if (p.test_stall == 1 && c == 0 && warp == 0 && wcount + n == 0) {
         mbar_arrive_expect_tx(bar, 16u);  // test hook: bytes that never arrive
       } else if (r.err == 0) {
         const size_t src = (size_t)r.pb * page_stride + head_off;

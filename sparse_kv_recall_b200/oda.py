@@ -50,6 +50,7 @@ ODA_STALL_NONE = 0
 ODA_STALL_DECODE_RING = 1
 ODA_STALL_LOCAL_CHAIN = 2
 ODA_STALL_FULL_CHAIN = 3
+ODA_STALL_LOCAL_PUSH = 4
 
 
 class OdaError(RuntimeError):

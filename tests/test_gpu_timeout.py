@@ -67,6 +67,28 @@ def test_decode_ring_wait_runs_out_then_recovers():
     assert_lse_close(lse.cpu().numpy(), rlse)
 
 
+def test_local_cluster_inbox_wait_runs_out_then_recovers():
+    """The per-layer Local cluster kernel (batch 1, eight KV heads: eight clusters): rank 1 of
+    the first cluster withholds its partial, so rank 0's wait for its inbox runs out (every
+    other partial has landed long before the 1 ms limit; the withholding CTA sends nothing),
+    the kernel returns with the status set; then a clean call matches the oracle."""
+    c = Case([3000], hq=16, hkv=8, seed=503)
+    out, lse = c.out_buffers()
+    with _Stall(oda.ODA_STALL_LOCAL_PUSH):
+        oda.oda_decode_local(c.kv, c.q, 4, 256, SCALE, out, c.ws, lse=lse)
+        torch.cuda.synchronize()
+    assert int(c.status.item()) == oda.ODA_DEV_TIMEOUT
+    c.status.zero_()
+    c.ws.zero_()
+    out, lse = c.out_buffers()
+    oda.oda_decode_local(c.kv, c.q, 4, 256, SCALE, out, c.ws, lse=lse)
+    torch.cuda.synchronize()
+    assert int(c.status.item()) == 0
+    ref, rlse = c.oracle(lambda b, t: O.local_positions(t, 4, 256))
+    assert_attn_close(out.cpu().numpy(), ref, "local after a timeout")
+    assert_lse_close(lse.cpu().numpy(), rlse)
+
+
 def _engine(w, lengths, theta, step_kernels=oda.ODA_STEP_PERSISTENT, **kw):
     lay = oda_synth.make_layout(w, extra_tokens=8, device="cuda", lengths=lengths)
     caches = [oda_synth.make_kv_cache(w, lay, l, device="cuda") for l in range(w.layers)]
