@@ -331,7 +331,13 @@ typedef struct {
   void* recall_ws;  size_t recall_ws_bytes;
   int32_t use_conditional;             /* 1: IF node around the Full phase; 0: Full kernels
                                           always launch and skip ungated sequences on-device */
-  int32_t timing_events;               /* 1: event-record nodes at phase boundaries          */
+  int32_t timing_events;               /* 1: event-record nodes at the four phase boundaries;
+                                          2: at the step's start and where the Full phase
+                                          starts and ends only (the Local-done and recall-done
+                                          events both where Full starts), so that the recall
+                                          head keeps its programmatic dependency on the last
+                                          Local layer (a graph without the recall phase records
+                                          Local-done after Local as with 1)                  */
   int32_t phases;                      /* 0 = whole step; else a mask of ODA_PHASE_* (a step
                                           without recall or Full is for measurement only)   */
   int32_t gate_source;                 /* ODA_GATE_RECALL: the recall head decides;

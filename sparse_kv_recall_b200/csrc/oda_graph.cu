@@ -25,6 +25,7 @@ struct oda_step_graph {
   cudaEvent_t placeholder[4] = {nullptr, nullptr, nullptr, nullptr};
   cudaGraphNode_t ev_node[4] = {nullptr, nullptr, nullptr, nullptr};
   bool timing = false;
+  int timing_mode = 0;          // desc->timing_events: 1 every phase boundary, 2 see oda.h
   int launches[3] = {0, 0, 0};  // kernels per step: Local, gate, Full
   oda::LocalChainPlan lplan;    // the persistent Local kernel's plan (decided before capture)
 };
@@ -94,7 +95,8 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
     if (rc != ODA_OK) return rc;
     ++g->launches[0];
   }
-  if (g->timing && (rc = record_event_node(g, 1)) != ODA_OK) return rc;
+  const bool lean_events = g->timing_mode == 2 && (phases & ODA_PHASE_RECALL);
+  if (g->timing && !lean_events && (rc = record_event_node(g, 1)) != ODA_OK) return rc;
   if (!(phases & ODA_PHASE_RECALL)) {
     if (g->timing)
       for (int i = 2; i < 4; ++i)
@@ -110,11 +112,12 @@ int capture_step(const oda_step_desc* d, oda_step_graph* g, cudaGraphConditional
       rc = oda::launch_recall(d->h_prev, d->emb, d->out[L - 1], ODA_F32, d->layers[0].batch,
                               hidden, d->mlp, d->w1, d->b1, d->w2, d->b2, d->theta, d->q_out,
                               d->gate_out, d->full_count, cond_u64, d->recall_ws,
-                              d->recall_ws_bytes, g->cap, g->timing ? 0 : 1);
+                              d->recall_ws_bytes, g->cap, g->timing && !lean_events ? 0 : 1);
     }
     if (rc != ODA_OK) return rc;
     g->launches[1] = 1;
   }
+  if (lean_events && (rc = record_event_node(g, 1)) != ODA_OK) return rc;
   if (g->timing && (rc = record_event_node(g, 2)) != ODA_OK) return rc;
 
   if (!(phases & ODA_PHASE_FULL)) {
@@ -204,6 +207,7 @@ int check_desc(const oda_step_desc* d) {
   if (d->step_kernels != ODA_STEP_FULL_PERSISTENT && d->step_kernels != ODA_STEP_PER_LAYER &&
       d->step_kernels != ODA_STEP_PERSISTENT)
     return ODA_ERR_INVALID_ARG;
+  if (d->timing_events < 0 || d->timing_events > 2) return ODA_ERR_INVALID_ARG;
   return ODA_OK;
 }
 
@@ -221,6 +225,7 @@ extern "C" int oda_step_graph_create(const oda_step_desc* desc, void* stream,
   oda_step_graph* g = new (std::nothrow) oda_step_graph();
   if (g == nullptr) return ODA_ERR_CUDA;
   g->timing = desc->timing_events != 0;
+  g->timing_mode = desc->timing_events;
   if (cudaStreamCreateWithFlags(&g->cap, cudaStreamNonBlocking) != cudaSuccess ||
       cudaStreamCreateWithFlags(&g->cap_body, cudaStreamNonBlocking) != cudaSuccess ||
       cudaGraphCreate(&g->graph, 0) != cudaSuccess) {

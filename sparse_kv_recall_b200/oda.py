@@ -384,7 +384,7 @@ class StepGraph:
                  h_prev, emb, w1, b1, w2, b2: float, theta: float, q_out, gate_out,
                  decode_ws, recall_ws, full_count=None, lse=None, local_layers=None,
                  sinks=None, windows=None, use_conditional: bool = True,
-                 timing_events: bool = False, phases: int = 0, gate_u=None, rho: float = 0.0,
+                 timing_events: int = 0, phases: int = 0, gate_u=None, rho: float = 0.0,
                  step_kernels: int = ODA_STEP_FULL_PERSISTENT):
         L = len(kvs)
         self._keep = []
@@ -424,7 +424,7 @@ class StepGraph:
             decode_ws_bytes=decode_ws.numel() * decode_ws.element_size(),
             recall_ws=_ptr(recall_ws, None, "recall_ws"),
             recall_ws_bytes=recall_ws.numel() * recall_ws.element_size(),
-            use_conditional=int(bool(use_conditional)), timing_events=int(bool(timing_events)),
+            use_conditional=int(bool(use_conditional)), timing_events=int(timing_events),
             phases=int(phases),
             gate_source=ODA_GATE_RANDOM if gate_u is not None else ODA_GATE_RECALL,
             gate_u=_ptr(gate_u, torch.float32, "gate_u"), rho=float(rho),

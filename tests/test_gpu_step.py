@@ -126,10 +126,14 @@ def test_step_graph_random_gate_schedule(use_conditional):
     assert 0 < n < 24
 
 
-def test_step_graph_with_timing_events():
+@pytest.mark.parametrize("mode", [1, 2])
+def test_step_graph_with_timing_events(mode):
+    """Event nodes at the four phase boundaries (mode 1), or at the step's start and around
+    the Full phase only (mode 2: the recall head stays programmatically dependent on the last
+    Local layer); either way the step decodes as the oracle does."""
     w = oda_synth.Workload(name="tiny3", layers=2, batch=2, num_q_heads=16, num_kv_heads=8,
                            prefill=700, steps=4, seed=79, sink=4, window=128)
-    _run_steps(w, [700, 300], 4, theta=0.0, timing=True)
+    _run_steps(w, [700, 300], 4, theta=0.0, timing=mode)
 
 
 def test_step_graph_all_local_and_all_full():
