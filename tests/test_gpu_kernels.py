@@ -84,11 +84,13 @@ def test_maximum_batch_local_and_full():
 @pytest.mark.parametrize("G,lens,sink,window", [
     (2, [1], 4, 2048), (2, [17], 4, 2048), (2, [2053], 4, 2048), (2, [40_000], 4, 2048),
     (1, [5000, 33], 4, 2048), (4, [9001, 2052], 0, 2100), (2, [700, 6000], 20, 100),
-    (2, [3000], 7, 33)])
+    (2, [3000], 7, 33), (2, [9000], 4, 2128), (4, [9000], 4, 2129)])
 def test_local_short_window_cluster_path(G, lens, sink, window):
     """Small batches take the cluster kernel for Local (one cluster per (sequence, KV head),
-    one page per warp, partials merged in distributed shared memory): outputs, normalisers,
-    attended rows and the fused commit against the oracle."""
+    one page per warp on cluster ranks 1-15, partials merged in rank 0's shared memory):
+    outputs, normalisers, attended rows and the fused commit against the oracle. Sink 4 with
+    window 2128 bounds the page list at the kernel's 135 pages; window 2129 (136) takes the
+    split kernel instead."""
     c = Case(lens, hq=8 * G, hkv=8, seed=90 + G + len(lens))
     out, lse = c.out_buffers()
     _run(c, lambda: oda.oda_decode_local(c.kv, c.q, sink, window, SCALE, out, c.ws,
