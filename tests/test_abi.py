@@ -209,7 +209,8 @@ def test_recall_training_argument_checks(lib):
 
 
 def test_step_desc_checks_before_any_cuda_call(lib):
-    """Per-layer access range, gate source and rho are validated on the host."""
+    """Per-layer access range, gate source, rho, the step-kernel mode and the timing-event
+    mode are validated on the host."""
     I = oda.ODA_ERR_INVALID_ARG
     L = 2
     kvs = (oda.oda_kv * L)(_kv(), _kv())
@@ -236,6 +237,7 @@ def test_step_desc_checks_before_any_cuda_call(lib):
     ints = lambda *v: ctypes.cast((ctypes.c_int32 * L)(*v), ctypes.POINTER(ctypes.c_int32))
     for d in [desc(sinks=ints(4, -1)), desc(windows=ints(0, 256)), desc(window=0),
               desc(gate_source=7), desc(gate_source=oda.ODA_GATE_RANDOM, gate_u=None, rho=0.5),
-              desc(gate_source=oda.ODA_GATE_RANDOM, gate_u=0x3000, rho=1.5)]:
+              desc(gate_source=oda.ODA_GATE_RANDOM, gate_u=0x3000, rho=1.5),
+              desc(step_kernels=3), desc(timing_events=3), desc(timing_events=-1)]:
         assert lib.oda_step_graph_create(ctypes.byref(d), None, ctypes.byref(h)) == I
         assert not h.value
