@@ -166,10 +166,11 @@ __global__ void __launch_bounds__(kLocalThreads, kLocalCtasPerSm)
     if (s_pages) atomicAdd(&p.stats[ODA_STAT_PAGES], s_pages);
   }
   cluster_wait();  // (long since complete: every CTA arrived at its start)
-  if (rank != 0 && !(p.test_stall == 2 && bg == 0 && rank == 1)) {
-    cluster_push_partial<G, kMma, kLocalWarps, false, true>(
-        m_run, l_run, acc, reinterpret_cast<float*>(stages), inbox, kPart, rank,
-        cluster_addr(&s_inbar, 0));
+  if (rank != 0) {
+    if (!(p.test_stall == 2 && bg == 0 && rank == 1))  // (test hook: withhold this partial)
+      cluster_push_partial<G, kMma, kLocalWarps, false, true>(
+          m_run, l_run, acc, reinterpret_cast<float*>(stages), inbox, kPart, rank,
+          cluster_addr(&s_inbar, 0));
   } else if (tid < kHeadDim) {
     if (!mbar_wait_cluster(&s_inbar, 0u, p.wait_ns)) {
       if (tid == 0) report(p.status, ODA_DEV_TIMEOUT);
